@@ -1,0 +1,148 @@
+"""fp64 CPU oracle of the MoBA causal prefill forward (ctypes wrapper of oracle.c).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU
+baseline leg may use it; the product path never does. It shares no code with
+the CUDA library. `oracle.c` lists each step with the page passage it follows.
+
+Inputs are host bf16 torch tensors in the [B, N, H, d] layout; results are
+float64 numpy arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so next to its source (gcc, OpenMP, no FP contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            lib.oracle_pool.restype = None
+            lib.oracle_pool.argtypes = [_P, _I, _I, _I, _I, _I, _P]
+            lib.oracle_select.restype = None
+            lib.oracle_select.argtypes = [_P, _P] + [_I] * 7 + [_P, _I, _P, _P, _P, _P, _I]
+            lib.oracle_attend.restype = _I
+            lib.oracle_attend.argtypes = [_P, _P, _P] + [_I] * 7 + [_P, _I, _P, _P, _P]
+            lib.oracle_attend_blockwise.restype = _I
+            lib.oracle_attend_blockwise.argtypes = [_P, _P, _P] + [_I] * 7 + [_P, _I, _P, _P, _P]
+            _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    if isinstance(a, torch.Tensor):
+        assert a.device.type == "cpu" and a.is_contiguous()
+        return a.data_ptr()
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def _check_bf16(*ts):
+    for t in ts:
+        assert isinstance(t, torch.Tensor) and t.dtype == torch.bfloat16 and t.device.type == "cpu"
+        assert t.is_contiguous() and t.dim() == 4
+
+
+def all_rows(B: int, Hq: int, N: int) -> np.ndarray:
+    """Every (b, hq, t) triple, b-major then head then token."""
+    b, h, t = np.meshgrid(np.arange(B), np.arange(Hq), np.arange(N), indexing="ij")
+    return np.ascontiguousarray(np.stack([b.ravel(), h.ravel(), t.ravel()], axis=1).astype(np.int64))
+
+
+def pool(k: torch.Tensor, block_size: int) -> np.ndarray:
+    """Kbar [B, Hkv, N // block_size, d]: the mean of each full key block, in fp64."""
+    _check_bf16(k)
+    B, N, Hkv, d = k.shape
+    nfull = N // block_size
+    kbar = np.zeros((B, Hkv, max(nfull, 1), d), dtype=np.float64)
+    _load().oracle_pool(_ptr(k), B, N, Hkv, d, block_size, _ptr(kbar))
+    return kbar[:, :, :nfull]
+
+
+def select(q: torch.Tensor, kbar: np.ndarray, Hkv: int, block_size: int, topk: int, rows: np.ndarray,
+           want_scores: bool = False):
+    """Selection of each row: (sel int32 [R, topk], s_last, s_next[, scores])."""
+    _check_bf16(q)
+    B, N, Hq, d = q.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    R = rows.shape[0]
+    nfull = N // block_size
+    kb = np.ascontiguousarray(kbar if kbar.shape[2] > 0 else np.zeros((B, Hkv, 1, d)), dtype=np.float64)
+    sel = np.empty((R, topk), dtype=np.int32)
+    s_last = np.empty(R, dtype=np.float64)
+    s_next = np.empty(R, dtype=np.float64)
+    max_past = max(nfull, 1)
+    scores = np.empty((R, max_past), dtype=np.float64) if want_scores else None
+    _load().oracle_select(_ptr(q), _ptr(kb), B, N, Hq, Hkv, d, block_size, topk, _ptr(rows), R,
+                          _ptr(sel), _ptr(s_last), _ptr(s_next),
+                          _ptr(scores) if want_scores else None, max_past)
+    if want_scores:
+        return sel, s_last, s_next, scores
+    return sel, s_last, s_next
+
+
+def attend(q, k, v, block_size: int, topk: int, rows: np.ndarray, sel: np.ndarray, blockwise: bool = False):
+    """(out [R, d], lse [R]) in fp64 for the rows with the given selection."""
+    _check_bf16(q, k, v)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    sel = np.ascontiguousarray(sel, dtype=np.int32)
+    R = rows.shape[0]
+    assert sel.shape == (R, topk)
+    out = np.zeros((R, d), dtype=np.float64)
+    lse = np.full(R, np.nan, dtype=np.float64)
+    fn = _load().oracle_attend_blockwise if blockwise else _load().oracle_attend
+    bad = fn(_ptr(q), _ptr(k), _ptr(v), B, N, Hq, Hkv, d, block_size, topk, _ptr(rows), R, _ptr(sel),
+             _ptr(out), _ptr(lse))
+    if bad:
+        raise ValueError(f"{bad} rows name a future block, repeat a block or lack their own block")
+    return out, lse
+
+
+def forward(q, k, v, block_size: int, topk: int, rows: np.ndarray | None = None):
+    """The whole method for the given rows (all rows by default).
+
+    Returns a dict with sel, s_last, s_next, out, lse (rows in the order given)."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if rows is None:
+        rows = all_rows(B, Hq, N)
+    kbar = pool(k, block_size)
+    sel, s_last, s_next = select(q, kbar, Hkv, block_size, topk, rows)
+    out, lse = attend(q, k, v, block_size, topk, rows, sel)
+    return {"rows": rows, "sel": sel, "s_last": s_last, "s_next": s_next, "out": out, "lse": lse}
+
+
+def near_tie(s_last: np.ndarray, s_next: np.ndarray, rel: float = 1e-5) -> np.ndarray:
+    """Rows whose last selected and first unselected past scores differ by < rel (relative)."""
+    a = np.abs(s_last - s_next)
+    m = np.maximum(np.abs(s_last), np.abs(s_next))
+    with np.errstate(invalid="ignore"):
+        return np.nan_to_num(a < rel * m, nan=False).astype(bool)
