@@ -1,0 +1,191 @@
+"""MoBA (Mixture of Block Attention) causal prefill forward on B200 (sm_100a).
+
+A thin Python binding over the C ABI of `libmoba.so` (declared in
+`include/moba.h`). This module only marshals arguments: it checks tensor
+dtypes, shapes and devices, takes device pointers and the current CUDA stream
+from PyTorch, and calls the library, where every step of the method runs in
+hand-written CUDA kernels. There is no CPU path: without the built library or a
+sm_100 device every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import flops  # noqa: F401  (work accounting helpers)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoba.so")
+
+MOBA_OK = 0
+STATUS_NAMES = {
+    0: "MOBA_OK", 1: "MOBA_ERR_NULL", 2: "MOBA_ERR_SHAPE", 3: "MOBA_ERR_ALIGN", 4: "MOBA_ERR_UNSUPPORTED",
+    5: "MOBA_ERR_CUDA", 6: "MOBA_ERR_OOM", 7: "MOBA_ERR_DEVICE_TIMEOUT", 8: "MOBA_ERR_WORKSPACE",
+    9: "MOBA_ERR_SELECTION",
+}
+
+EXPORTED = [
+    "moba_status_string", "moba_workspace_size", "moba_forward", "moba_forward_ws", "moba_gate",
+    "moba_forward_selected", "moba_forward_selected_ws", "moba_dense_causal", "moba_sync_status",
+    "moba_set_attention_impl", "moba_set_gate_impl",
+]
+
+
+class MobaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({_status_string(status)})")
+
+
+_lock = threading.Lock()
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_L = ctypes.c_int64
+
+
+def lib():
+    """The loaded libmoba.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"libmoba.so is missing at {LIB_PATH}; build it with "
+                                   "block_sparse_long_gate_b200.build.build_library()")
+            L = ctypes.CDLL(LIB_PATH)
+            L.moba_status_string.restype = ctypes.c_char_p
+            L.moba_status_string.argtypes = [_I]
+            L.moba_workspace_size.restype = _I
+            L.moba_workspace_size.argtypes = [_I, _I, _I, _L, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]
+            L.moba_forward.restype = _I
+            L.moba_forward.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P]
+            L.moba_forward_ws.restype = _I
+            L.moba_forward_ws.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P, ctypes.c_size_t, _P]
+            L.moba_gate.restype = _I
+            L.moba_gate.argtypes = [_P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P]
+            L.moba_forward_selected.restype = _I
+            L.moba_forward_selected.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P]
+            L.moba_forward_selected_ws.restype = _I
+            L.moba_forward_selected_ws.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P,
+                                                   ctypes.c_size_t, _P]
+            L.moba_dense_causal.restype = _I
+            L.moba_dense_causal.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _L, _I, _P]
+            L.moba_sync_status.restype = _I
+            L.moba_sync_status.argtypes = [_P]
+            L.moba_set_attention_impl.restype = _I
+            L.moba_set_attention_impl.argtypes = [_I]
+            L.moba_set_gate_impl.restype = _I
+            L.moba_set_gate_impl.argtypes = [_I]
+            _lib = L
+    return _lib
+
+
+def _status_string(status: int) -> str:
+    try:
+        return lib().moba_status_string(status).decode()
+    except Exception:  # library not loadable: fall back to the name table
+        return STATUS_NAMES.get(status, "unknown")
+
+
+def _check(status: int, where: str):
+    if status != MOBA_OK:
+        raise MobaError(status, where)
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _check_qkv(q, k, v=None):
+    ts = [q, k] + ([v] if v is not None else [])
+    for t in ts:
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+        if t.dim() != 4:
+            raise ValueError("q, k, v must have the layout [B, N, H, d]")
+    B, N, Hq, d = q.shape
+    if k.shape[0] != B or k.shape[1] != N or k.shape[3] != d:
+        raise ValueError("k must be [B, N, Hkv, d] matching q")
+    if v is not None and v.shape != k.shape:
+        raise ValueError("v must have the shape of k")
+    return B, N, Hq, k.shape[2], d
+
+
+def workspace_size(B, Hq, Hkv, N, d, block_size, topk) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moba_workspace_size(B, Hq, Hkv, N, d, block_size, topk, ctypes.byref(n)), "moba_workspace_size")
+    return int(n.value)
+
+
+def forward(q, k, v, block_size: int, topk: int, out=None, lse=None, workspace=None, stream=None):
+    """MoBA causal prefill forward. Returns (out bf16 [B, N, Hq, d], lse fp32 [B, Hq, N])."""
+    B, N, Hq, Hkv, d = _check_qkv(q, k, v)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    if workspace is None:
+        workspace = torch.empty(workspace_size(B, Hq, Hkv, N, d, block_size, topk), dtype=torch.uint8,
+                                device=q.device)
+    _check(lib().moba_forward_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d, block_size,
+                                 topk, _ptr(workspace), workspace.numel(), _stream(stream)), "moba_forward_ws")
+    return out, lse
+
+
+def gate(q, k, block_size: int, topk: int, idx=None, stream=None):
+    """Selected blocks per query: int32 [B, Hq, N, topk], ascending, own block last, -1 padded."""
+    B, N, Hq, Hkv, d = _check_qkv(q, k)
+    idx = torch.empty((B, Hq, N, topk), dtype=torch.int32, device=q.device) if idx is None else idx
+    _check(lib().moba_gate(_ptr(q), _ptr(k), _ptr(idx), B, Hq, Hkv, N, d, block_size, topk, _stream(stream)),
+           "moba_gate")
+    return idx
+
+
+def forward_selected(q, k, v, idx, block_size: int, topk: int, out=None, lse=None, workspace=None, stream=None):
+    """Attention with a given selection (same layout as gate()). Returns (out, lse)."""
+    B, N, Hq, Hkv, d = _check_qkv(q, k, v)
+    if idx.dtype != torch.int32 or not idx.is_cuda or not idx.is_contiguous() or tuple(idx.shape) != (B, Hq, N, topk):
+        raise ValueError("idx must be a contiguous int32 CUDA tensor [B, Hq, N, topk]")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    if workspace is None:
+        workspace = torch.empty(workspace_size(B, Hq, Hkv, N, d, block_size, topk), dtype=torch.uint8,
+                                device=q.device)
+    _check(lib().moba_forward_selected_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(out), _ptr(lse), B, Hq, Hkv,
+                                          N, d, block_size, topk, _ptr(workspace), workspace.numel(),
+                                          _stream(stream)), "moba_forward_selected_ws")
+    return out, lse
+
+
+def dense_causal(q, k, v, out=None, lse=None, stream=None):
+    """Dense causal attention of the same shape. Returns (out, lse)."""
+    B, N, Hq, Hkv, d = _check_qkv(q, k, v)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(lib().moba_dense_causal(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
+                                   _stream(stream)), "moba_dense_causal")
+    return out, lse
+
+
+def sync_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the library's device error flag."""
+    return int(lib().moba_sync_status(_stream(stream)))
+
+
+def check_status(stream=None):
+    _check(sync_status(stream), "device")
+
+
+def set_attention_impl(impl: int) -> int:
+    return int(lib().moba_set_attention_impl(impl))
+
+
+def set_gate_impl(impl: int) -> int:
+    return int(lib().moba_set_gate_impl(impl))

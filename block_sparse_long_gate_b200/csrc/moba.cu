@@ -1,0 +1,389 @@
+// moba.cu - the C ABI of libmoba: argument checks, workspace layout and the
+// launch sequence of the MoBA causal prefill forward on one sm_100a GPU.
+//
+//   pool (K -> Kbar) -> gate (Q, Kbar -> idx) -> count / scan / scatter
+//   (idx -> per-block query lists) -> attention tiles (past blocks -> partials,
+//   own block -> out / lse) -> merge (partials -> out / lse)
+//
+// Everything after the host-side checks is queued on the caller's stream; no
+// call synchronises the device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "common.cuh"
+#include "k_attn_common.cuh"
+#include "k_attn_simt.cuh"
+#include "k_attn_tc.cuh"
+#include "k_gate.cuh"
+#include "k_invert.cuh"
+#include "k_merge.cuh"
+#include "k_pool.cuh"
+
+namespace {
+
+int g_attn_impl = 1;  // 0 tensor cores, 1 CUDA cores
+int g_gate_impl = 0;
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Plan {
+    int B, Hq, Hkv, G, d, bs, topk, kp;
+    int64_t N, nblk, nfull, L, nch, E, Pmax, D, mb, ml, per_bh, nseg, nscan_parts;
+    size_t off_kbar, off_idx, off_counts, off_segoff, off_tiles, off_parts, off_entries, off_opart, off_lpart;
+    size_t total;
+};
+
+int make_plan(int B, int Hq, int Hkv, int64_t N, int d, int bs, int topk, Plan* p) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || bs < 1 || topk < 1) return MOBA_ERR_SHAPE;
+    if (d != MOBA_D || Hq % Hkv != 0 || topk > MOBA_MAX_TOPK || N >= ((int64_t)1 << 31)) return MOBA_ERR_SHAPE;
+    if (B > 65535 || Hq > 65535) return MOBA_ERR_SHAPE;
+    Plan& P = *p;
+    P.B = B;
+    P.Hq = Hq;
+    P.Hkv = Hkv;
+    P.G = Hq / Hkv;
+    P.d = d;
+    P.bs = bs;
+    P.topk = topk;
+    P.kp = topk - 1;
+    P.N = N;
+    P.nblk = cdiv(N, bs);
+    if (P.nblk > MOBA_MAX_BLOCKS) return MOBA_ERR_SHAPE;  // per-block counters live in shared memory
+    P.nfull = N / bs;
+    P.L = (int64_t)B * Hkv * P.nblk;
+    P.nch = cdiv(N, INV_CHUNK);
+    // exact number of earlier-block selections of well-formed rows: sum_t min(c(t), k - 1)
+    int64_t per_head = 0;
+    for (int64_t c = 0; c < P.nblk; ++c) {
+        int64_t n_c = (c * bs + bs <= N) ? bs : N - c * bs;
+        per_head += n_c * (c < P.kp ? c : P.kp);
+    }
+    P.E = per_head * B * Hq;
+    P.Pmax = P.E / MOBA_TILE + P.L;
+    P.mb = cdiv(bs, MOBA_TILE);
+    int64_t nlast = N - (P.nblk - 1) * bs;
+    P.ml = cdiv(nlast, MOBA_TILE);
+    P.per_bh = (P.nblk - 1) * P.mb + P.ml;
+    P.D = (int64_t)B * Hq * P.per_bh;
+    P.nseg = P.L * P.nch;
+    int64_t nscan = P.nseg > P.L ? P.nseg : P.L;
+    P.nscan_parts = cdiv(nscan, SCAN_TILE);
+
+    size_t o = 0;
+    P.off_kbar = o;
+    o = align256(o + sizeof(double) * (size_t)B * Hkv * (P.nfull > 0 ? P.nfull : 1) * MOBA_D);
+    P.off_idx = o;
+    o = align256(o + sizeof(int32_t) * (size_t)B * Hq * N * topk);
+    P.off_counts = o;
+    o = align256(o + sizeof(uint32_t) * (size_t)P.nseg);
+    P.off_segoff = o;
+    o = align256(o + sizeof(int64_t) * (size_t)(P.nseg + 1));
+    P.off_tiles = o;
+    o = align256(o + sizeof(int64_t) * (size_t)(P.L + 1));
+    P.off_parts = o;
+    o = align256(o + sizeof(int64_t) * (size_t)P.nscan_parts);
+    P.off_entries = o;
+    o = align256(o + sizeof(uint64_t) * (size_t)(P.E > 0 ? P.E : 1));
+    P.off_opart = o;
+    o = align256(o + sizeof(uint16_t) * (size_t)B * Hq * N * (P.kp > 0 ? P.kp : 1) * MOBA_D);
+    P.off_lpart = o;
+    o = align256(o + sizeof(float) * (size_t)B * Hq * N * (P.kp > 0 ? P.kp : 1));
+    P.total = o;
+    return MOBA_OK;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+int check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOBA_ERR_CUDA;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MOBA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return MOBA_ERR_CUDA;
+    if (major != 10 || minor != 0) return MOBA_ERR_UNSUPPORTED;
+    return MOBA_OK;
+}
+
+int check_ptrs(std::initializer_list<const void*> ps) {
+    for (const void* p : ps)
+        if (!p) return MOBA_ERR_NULL;
+    for (const void* p : ps)
+        if (!aligned16(p)) return MOBA_ERR_ALIGN;
+    return MOBA_OK;
+}
+
+int launch_ok() { return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA; }
+
+// ---------------------------------------------------------------- stages
+int run_pool(const Plan& P, const void* k, double* kbar, cudaStream_t st) {
+    if (P.nfull == 0) return MOBA_OK;
+    dim3 grid((unsigned)P.nfull, P.Hkv, P.B);
+    moba_pool_kernel<<<grid, POOL_THREADS, 0, st>>>((const uint16_t*)k, kbar, P.N, P.Hkv, P.bs, P.nfull);
+    return launch_ok();
+}
+
+int run_gate(const Plan& P, const void* q, const double* kbar, int32_t* idx, cudaStream_t st) {
+    dim3 grid((unsigned)cdiv(P.N, GATE_ROWS), P.Hq, P.B);
+    const uint16_t* qq = (const uint16_t*)q;
+    if (P.kp <= 8)
+        moba_gate_simt_kernel<8><<<grid, GATE_ROWS, 0, st>>>(qq, kbar, idx, P.N, P.Hq, P.Hkv, P.bs, P.topk, P.nfull);
+    else if (P.kp <= 16)
+        moba_gate_simt_kernel<16><<<grid, GATE_ROWS, 0, st>>>(qq, kbar, idx, P.N, P.Hq, P.Hkv, P.bs, P.topk, P.nfull);
+    else if (P.kp <= 32)
+        moba_gate_simt_kernel<32><<<grid, GATE_ROWS, 0, st>>>(qq, kbar, idx, P.N, P.Hq, P.Hkv, P.bs, P.topk, P.nfull);
+    else
+        moba_gate_simt_kernel<64><<<grid, GATE_ROWS, 0, st>>>(qq, kbar, idx, P.N, P.Hq, P.Hkv, P.bs, P.topk, P.nfull);
+    return launch_ok();
+}
+
+int run_scan(ScanSrc src, int64_t n, int64_t* parts, int64_t* out, cudaStream_t st) {
+    int64_t nb = cdiv(n, SCAN_TILE);
+    moba_scan_partial_kernel<<<(unsigned)nb, SCAN_THREADS, 0, st>>>(src, n, parts);
+    moba_scan_top_kernel<<<1, SCAN_THREADS, 0, st>>>(parts, nb);
+    moba_scan_final_kernel<<<(unsigned)nb, SCAN_THREADS, 0, st>>>(src, n, parts, out);
+    return launch_ok();
+}
+
+int run_invert(const Plan& P, const int32_t* idx, char* ws, cudaStream_t st) {
+    uint32_t* counts = (uint32_t*)(ws + P.off_counts);
+    int64_t* segoff = (int64_t*)(ws + P.off_segoff);
+    int64_t* tiles = (int64_t*)(ws + P.off_tiles);
+    int64_t* parts = (int64_t*)(ws + P.off_parts);
+    uint64_t* entries = (uint64_t*)(ws + P.off_entries);
+    dim3 grid((unsigned)P.nch, P.Hkv, P.B);
+    size_t sm_count = sizeof(uint32_t) * (size_t)P.nblk;
+    size_t sm_scatter = (sizeof(int64_t) + sizeof(uint32_t)) * (size_t)P.nblk;
+    if (cudaFuncSetAttribute(moba_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_count) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(moba_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_scatter) !=
+            cudaSuccess)
+        return MOBA_ERR_CUDA;
+    moba_count_kernel<<<grid, INV_THREADS, sm_count, st>>>(idx, counts, P.N, P.Hq, P.Hkv, P.bs, P.topk, P.nblk,
+                                                           P.nch);
+    int rc = launch_ok();
+    if (rc) return rc;
+    ScanSrc s1{counts, nullptr, 0};
+    if ((rc = run_scan(s1, P.nseg, parts, segoff, st))) return rc;
+    ScanSrc s2{nullptr, segoff, P.nch};
+    if ((rc = run_scan(s2, P.L, parts, tiles, st))) return rc;
+    moba_scatter_kernel<<<grid, INV_THREADS, sm_scatter, st>>>(idx, segoff, entries, P.N, P.Hq, P.Hkv, P.bs,
+                                                               P.topk, P.nblk, P.nch);
+    return launch_ok();
+}
+
+AttnParams attn_params(const Plan& P, const void* q, const void* k, const void* v, void* out, float* lse,
+                       char* ws) {
+    AttnParams a;
+    a.q = (const uint16_t*)q;
+    a.k = (const uint16_t*)k;
+    a.v = (const uint16_t*)v;
+    a.N = P.N;
+    a.B = P.B;
+    a.Hq = P.Hq;
+    a.Hkv = P.Hkv;
+    a.G = P.G;
+    a.bs = P.bs;
+    a.topk = P.topk;
+    a.kp = P.kp;
+    a.nblk = P.nblk;
+    a.nch = P.nch;
+    a.entries = ws ? (const uint64_t*)(ws + P.off_entries) : nullptr;
+    a.segoff = ws ? (const int64_t*)(ws + P.off_segoff) : nullptr;
+    a.tile_start = ws ? (const int64_t*)(ws + P.off_tiles) : nullptr;
+    a.L = P.L;
+    a.Pmax = P.Pmax;
+    a.opart = ws ? (uint16_t*)(ws + P.off_opart) : nullptr;
+    a.lpart = ws ? (float*)(ws + P.off_lpart) : nullptr;
+    a.D = P.D;
+    a.mb = P.mb;
+    a.ml = P.ml;
+    a.per_bh = P.per_bh;
+    a.dense = 0;
+    a.out = (uint16_t*)out;
+    a.lse = lse;
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)P.d));
+    return a;
+}
+
+int run_attention(const Plan& P, const AttnParams& a, cudaStream_t st) {
+    const int64_t items = a.Pmax + a.D;
+    if (g_attn_impl == 1) {
+        for (int64_t i0 = 0; i0 < items; i0 += (int64_t)1 << 30) {
+            int64_t n = items - i0 < ((int64_t)1 << 30) ? items - i0 : ((int64_t)1 << 30);
+            moba_attn_simt_kernel<<<(unsigned)n, 128, 0, st>>>(a, i0);
+        }
+        return launch_ok();
+    }
+    return run_attention_tc(a, st);
+}
+
+int run_merge(const Plan& P, const int32_t* idx, char* ws, void* out, float* lse, cudaStream_t st) {
+    int64_t nrows = (int64_t)P.B * P.Hq * P.N;
+    moba_merge_kernel<<<(unsigned)cdiv(nrows, 8), 256, 0, st>>>(
+        idx, (const uint16_t*)(ws + P.off_opart), (const float*)(ws + P.off_lpart), (uint16_t*)out, lse, P.N, P.Hq,
+        P.bs, P.topk, nrows);
+    return launch_ok();
+}
+
+int forward_impl(const void* q, const void* k, const void* v, const int32_t* idx_in, void* out, float* lse,
+                 int B, int Hq, int Hkv, int64_t N, int d, int bs, int topk, void* ws_ptr, size_t ws_bytes,
+                 cudaStream_t st) {
+    Plan P;
+    int rc = make_plan(B, Hq, Hkv, N, d, bs, topk, &P);
+    if (rc) return rc;
+    if ((rc = check_ptrs({q, k, v, out, lse}))) return rc;
+    if (idx_in && !aligned16(idx_in)) return MOBA_ERR_ALIGN;
+    if ((rc = check_device())) return rc;
+    bool own = false;
+    char* ws = (char*)ws_ptr;
+    if (!ws) {
+        if (cudaMallocAsync((void**)&ws, P.total, st) != cudaSuccess) {
+            cudaGetLastError();
+            return MOBA_ERR_OOM;
+        }
+        own = true;
+    } else if (ws_bytes < P.total || ((uintptr_t)ws & 255)) {
+        return MOBA_ERR_WORKSPACE;
+    }
+    const int32_t* idx = idx_in;
+    do {
+        if (!idx) {
+            int32_t* widx = (int32_t*)(ws + P.off_idx);
+            if ((rc = run_pool(P, k, (double*)(ws + P.off_kbar), st))) break;
+            if ((rc = run_gate(P, q, (const double*)(ws + P.off_kbar), widx, st))) break;
+            idx = widx;
+        }
+        if ((rc = run_invert(P, idx, ws, st))) break;
+        AttnParams a = attn_params(P, q, k, v, out, lse, ws);
+        if ((rc = run_attention(P, a, st))) break;
+        if ((rc = run_merge(P, idx, ws, out, lse, st))) break;
+    } while (0);
+    if (own) cudaFreeAsync(ws, st);
+    return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moba_status_string(int s) {
+    switch (s) {
+        case MOBA_OK: return "ok";
+        case MOBA_ERR_NULL: return "null pointer";
+        case MOBA_ERR_SHAPE: return "unsupported sizes";
+        case MOBA_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case MOBA_ERR_UNSUPPORTED: return "device is not sm_100";
+        case MOBA_ERR_CUDA: return "CUDA error";
+        case MOBA_ERR_OOM: return "workspace allocation failed";
+        case MOBA_ERR_DEVICE_TIMEOUT: return "device wait reached its limit";
+        case MOBA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+        case MOBA_ERR_SELECTION: return "malformed selection row";
+        default: return "unknown status";
+    }
+}
+
+int moba_workspace_size(int B, int Hq, int Hkv, int64_t N, int d, int block_size, int topk, size_t* bytes) {
+    if (!bytes) return MOBA_ERR_NULL;
+    Plan P;
+    int rc = make_plan(B, Hq, Hkv, N, d, block_size, topk, &P);
+    if (rc) return rc;
+    *bytes = P.total;
+    return MOBA_OK;
+}
+
+int moba_forward(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                 int64_t N, int d, int block_size, int topk, moba_stream_t stream) {
+    return forward_impl(q, k, v, nullptr, out, lse, B, Hq, Hkv, N, d, block_size, topk, nullptr, 0,
+                        (cudaStream_t)stream);
+}
+
+int moba_forward_ws(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                    int64_t N, int d, int block_size, int topk, void* workspace, size_t workspace_bytes,
+                    moba_stream_t stream) {
+    if (!workspace) return MOBA_ERR_WORKSPACE;
+    return forward_impl(q, k, v, nullptr, out, lse, B, Hq, Hkv, N, d, block_size, topk, workspace,
+                        workspace_bytes, (cudaStream_t)stream);
+}
+
+int moba_forward_selected(const void* q, const void* k, const void* v, const int32_t* idx, void* out, float* lse,
+                          int B, int Hq, int Hkv, int64_t N, int d, int block_size, int topk,
+                          moba_stream_t stream) {
+    if (!idx) return MOBA_ERR_NULL;
+    return forward_impl(q, k, v, idx, out, lse, B, Hq, Hkv, N, d, block_size, topk, nullptr, 0,
+                        (cudaStream_t)stream);
+}
+
+int moba_forward_selected_ws(const void* q, const void* k, const void* v, const int32_t* idx, void* out,
+                             float* lse, int B, int Hq, int Hkv, int64_t N, int d, int block_size, int topk,
+                             void* workspace, size_t workspace_bytes, moba_stream_t stream) {
+    if (!idx) return MOBA_ERR_NULL;
+    if (!workspace) return MOBA_ERR_WORKSPACE;
+    return forward_impl(q, k, v, idx, out, lse, B, Hq, Hkv, N, d, block_size, topk, workspace, workspace_bytes,
+                        (cudaStream_t)stream);
+}
+
+int moba_gate(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv, int64_t N, int d,
+              int block_size, int topk, moba_stream_t stream) {
+    Plan P;
+    int rc = make_plan(B, Hq, Hkv, N, d, block_size, topk, &P);
+    if (rc) return rc;
+    if ((rc = check_ptrs({q, k, (const void*)idx}))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    double* kbar = nullptr;
+    size_t kb_bytes = sizeof(double) * (size_t)B * Hkv * (P.nfull > 0 ? P.nfull : 1) * MOBA_D;
+    if (cudaMallocAsync((void**)&kbar, kb_bytes, st) != cudaSuccess) {
+        cudaGetLastError();
+        return MOBA_ERR_OOM;
+    }
+    rc = run_pool(P, k, kbar, st);
+    if (!rc) rc = run_gate(P, q, kbar, idx, st);
+    cudaFreeAsync(kbar, st);
+    return rc;
+}
+
+int moba_dense_causal(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                      int64_t N, int d, moba_stream_t stream) {
+    Plan P;
+    if (N < 1 || N >= ((int64_t)1 << 31)) return MOBA_ERR_SHAPE;
+    int rc = make_plan(B, Hq, Hkv, N, d, (int)N, 1, &P);
+    if (rc) return rc;
+    if ((rc = check_ptrs({q, k, v, out, lse}))) return rc;
+    if ((rc = check_device())) return rc;
+    AttnParams a = attn_params(P, q, k, v, out, lse, nullptr);
+    a.dense = 1;
+    a.Pmax = 0;
+    a.L = 0;
+    return run_attention(P, a, (cudaStream_t)stream);
+}
+
+int moba_sync_status(moba_stream_t stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
+        cudaGetLastError();
+        return MOBA_ERR_CUDA;
+    }
+    int flag = 0;
+    if (cudaMemcpyFromSymbol(&flag, g_moba_err, sizeof(int)) != cudaSuccess) return MOBA_ERR_CUDA;
+    if (flag) {
+        int zero = 0;
+        if (cudaMemcpyToSymbol(g_moba_err, &zero, sizeof(int)) != cudaSuccess) return MOBA_ERR_CUDA;
+    }
+    return flag;
+}
+
+int moba_set_attention_impl(int impl) {
+    int old = g_attn_impl;
+    g_attn_impl = impl;
+    return old;
+}
+
+int moba_set_gate_impl(int impl) {
+    int old = g_gate_impl;
+    g_gate_impl = impl;
+    return old;
+}
+
+}  // extern "C"

@@ -1,0 +1,144 @@
+/*
+ * moba.h - C ABI of libmoba, the sm_100a (B200) implementation of the causal
+ * prefill forward of MoBA (Mixture of Block Attention).
+ *
+ * The method (sources: "MoBA project hub" page, Steps 1-3; "MoBA tech-report
+ * summary" page, section 2; "KIMI MoBA" blog, section 3 configuration fields;
+ * "NSA vs MoBA" blog, section 1 attention formula):
+ *   - keys are cut into blocks of block_size consecutive tokens; token t lies
+ *     in block c(t) = floor(t / block_size);
+ *   - each full block j is represented by the mean of its keys, Kbar_j;
+ *   - query t scores every earlier block j < c(t) as <q_t, Kbar_j> (no gate
+ *     parameters, no scaling), always keeps its own block c(t), and keeps the
+ *     topk - 1 best earlier blocks (higher score first, lower block index on
+ *     equal scores); with c(t) <= topk - 1 every earlier block is kept;
+ *   - it attends with softmax(q k^T / sqrt(d)) over all keys of the kept
+ *     earlier blocks plus the keys c(t) * block_size .. t of its own block; the
+ *     per-block partial results are merged by log-sum-exp.
+ *
+ * Conventions for every entry point:
+ *   - q, out: bf16 [B, N, Hq, d]; k, v: bf16 [B, N, Hkv, d]; all contiguous.
+ *     Query head h uses kv head floor(h / (Hq / Hkv)) (grouped-query sharing).
+ *   - lse: fp32 [B, Hq, N], natural log of the softmax denominator of the
+ *     scaled logits q.k / sqrt(d).
+ *   - idx: int32 [B, Hq, N, topk], the kept blocks of each query in ascending
+ *     order (so the own block c(t) comes last), padded with -1 when fewer than
+ *     topk blocks exist.
+ *   - All pointers are DEVICE pointers owned by the caller, 16-byte aligned.
+ *     The library never frees or keeps them after the call returns.
+ *   - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default stream)
+ *     and runs asynchronously; an entry point returns once its work is queued.
+ *   - Arguments are validated on the host before anything is queued; an invalid
+ *     call returns a status code and queues nothing.
+ *   - Asynchronous failures (a kernel wait that hit its iteration limit, a
+ *     launch error) are reported by moba_sync_status().
+ *   - Supported: d = 128, Hq % Hkv == 0, 1 <= topk <= 64, block_size >= 1,
+ *     1 <= N < 2^31, ceil(N / block_size) <= 16384, B and Hq <= 65535, and a
+ *     device of compute capability 10.0 (sm_100a).
+ */
+#ifndef MOBA_H
+#define MOBA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t, declared here so the header needs no CUDA include. */
+typedef struct CUstream_st* moba_stream_t;
+
+typedef enum {
+    MOBA_OK = 0,
+    MOBA_ERR_NULL = 1,           /* a required pointer is NULL */
+    MOBA_ERR_SHAPE = 2,          /* unsupported sizes (see the list above) */
+    MOBA_ERR_ALIGN = 3,          /* a pointer is not 16-byte aligned */
+    MOBA_ERR_UNSUPPORTED = 4,    /* the current device is not sm_100 */
+    MOBA_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
+    MOBA_ERR_OOM = 6,            /* the internal workspace could not be allocated */
+    MOBA_ERR_DEVICE_TIMEOUT = 7, /* a kernel gave up waiting (bounded wait hit its limit) */
+    MOBA_ERR_WORKSPACE = 8,      /* the caller's workspace is NULL or too small */
+    MOBA_ERR_SELECTION = 9       /* an injected selection is malformed (found on the device) */
+} moba_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moba_status_string(int status);
+
+/*
+ * Bytes of device workspace moba_forward_ws() needs for these sizes
+ * (block mean keys, selection, per-block query lists and per-slot partial
+ * outputs). Writes the count to *bytes. No device work.
+ */
+int moba_workspace_size(int B, int Hq, int Hkv, int64_t N, int d, int block_size, int topk,
+                        size_t* bytes);
+
+/*
+ * The whole causal prefill forward: pooling, gating, top-k with the forced own
+ * block, selection inversion, block-sparse attention and log-sum-exp merge.
+ * Writes out and lse. Allocates its workspace with cudaMallocAsync on `stream`
+ * and frees it on the same stream.
+ */
+int moba_forward(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                 int Hkv, int64_t N, int d, int block_size, int topk, moba_stream_t stream);
+
+/* moba_forward with a caller-owned device workspace of at least moba_workspace_size() bytes
+ * (256-byte aligned). The workspace must not be used by other work until the call's
+ * stream work has finished. */
+int moba_forward_ws(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                    int Hkv, int64_t N, int d, int block_size, int topk, void* workspace,
+                    size_t workspace_bytes, moba_stream_t stream);
+
+/*
+ * Gating only: block mean pooling, scores <q_t, Kbar_j> over earlier blocks,
+ * forced own block and top-k. Writes idx (int32 [B, Hq, N, topk]).
+ * Allocates its small scratch (the block means) with cudaMallocAsync on `stream`.
+ */
+int moba_gate(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv, int64_t N, int d,
+              int block_size, int topk, moba_stream_t stream);
+
+/*
+ * Attention with a given selection idx (same layout as moba_gate's output):
+ * selection inversion, block-sparse attention and merge. Each row must list
+ * distinct blocks <= c(t) and include c(t); a malformed row is skipped and
+ * reported as MOBA_ERR_SELECTION by moba_sync_status(). Allocates its
+ * workspace with cudaMallocAsync on `stream`.
+ */
+int moba_forward_selected(const void* q, const void* k, const void* v, const int32_t* idx, void* out,
+                          float* lse, int B, int Hq, int Hkv, int64_t N, int d, int block_size,
+                          int topk, moba_stream_t stream);
+
+/* moba_forward_selected with a caller-owned workspace of at least moba_workspace_size() bytes. */
+int moba_forward_selected_ws(const void* q, const void* k, const void* v, const int32_t* idx,
+                             void* out, float* lse, int B, int Hq, int Hkv, int64_t N, int d,
+                             int block_size, int topk, void* workspace, size_t workspace_bytes,
+                             moba_stream_t stream);
+
+/*
+ * Dense causal softmax attention of the same shape (every key u <= t), the
+ * comparison point of the method's speedup figures ("MoBA tech-report summary",
+ * section 3). Writes out and lse. Needs no workspace.
+ */
+int moba_dense_causal(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                      int Hkv, int64_t N, int d, moba_stream_t stream);
+
+/*
+ * Waits for `stream`, then returns and clears the library's device-side error
+ * flag on the current device (MOBA_OK if no kernel reported a failure), or
+ * MOBA_ERR_CUDA if the stream reported a CUDA error.
+ */
+int moba_sync_status(moba_stream_t stream);
+
+/* Implementation selector for the attention step: 0 = tensor-core kernel (default),
+ * 1 = the simple CUDA-core kernel kept as a cross-check. Returns the previous value. */
+int moba_set_attention_impl(int impl);
+
+/* Implementation selector for the gate: 0 = default, 1 = the CUDA-core fp64 kernel.
+ * Returns the previous value. */
+int moba_set_gate_impl(int impl);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOBA_H */

@@ -21,3 +21,24 @@ def _build_host_libs():
     synth.build()
     oracle.build()
     yield
+
+
+@pytest.fixture(scope="session")
+def moba():
+    """The package with libmoba.so built in-tree."""
+    from block_sparse_long_gate_b200.build import build_library
+
+    build_library()
+    import block_sparse_long_gate_b200 as m
+
+    m.lib()
+    return m
+
+
+@pytest.fixture(scope="session")
+def cuda_dev():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    return torch.device("cuda:0")

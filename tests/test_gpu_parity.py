@@ -1,0 +1,150 @@
+"""GPU parity: libmoba (through its C ABI) against the fp64 oracle on the same seeded inputs.
+
+Selections must match bit for bit, except at near ties: rows whose oracle
+(k-1)-th and k-th past scores differ by < 1e-5 relative. Those rows are
+re-checked with the oracle's selection injected. Outputs must be within
+max-abs 2e-2 and mean-abs 2e-3 (bf16 I/O) and lse within 1e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+OUT_MAX, OUT_MEAN, LSE_MAX = 2e-2, 2e-3, 1e-3
+
+
+def _inputs(B, N, Hq, Hkv, bs, seed, dev):
+    q, k, v = synth.inputs(B, N, Hq, Hkv, 128, bs, seed)
+    return (q, k, v), (q.to(dev), k.to(dev), v.to(dev))
+
+
+def sample_rows(B, Hq, N, bs, topk, per_head=256, seed=0):
+    """Seeded rows per (b, hq): random tokens plus block edges, the first and last block
+    and the rows with c <= k - 1."""
+    rng = np.random.default_rng(seed)
+    special = {0, N - 1, min(bs - 1, N - 1), min(bs, N - 1), min((topk - 1) * bs, N - 1),
+               min(topk * bs, N - 1), min(max(topk * bs - 1, 0), N - 1), N // 2}
+    rows = []
+    for b in range(B):
+        for h in range(Hq):
+            ts = set(rng.integers(0, N, size=min(per_head, N)).tolist()) | special
+            rows += [(b, h, t) for t in sorted(ts)]
+    return np.array(rows, dtype=np.int64)
+
+
+def _gather(gpu_out, gpu_lse, rows):
+    o = gpu_out.float().cpu().numpy()
+    l = gpu_lse.cpu().numpy()
+    return o[rows[:, 0], rows[:, 2], rows[:, 1]], l[rows[:, 0], rows[:, 1], rows[:, 2]]
+
+
+def _compare_outputs(out, lse, ref_out, ref_lse, what=""):
+    err = np.abs(out.astype(np.float64) - ref_out)
+    lerr = np.abs(lse.astype(np.float64) - ref_lse)
+    assert np.isfinite(out).all() and np.isfinite(lse).all(), what
+    assert err.max() <= OUT_MAX, (what, err.max())
+    assert err.mean() <= OUT_MEAN, (what, err.mean())
+    assert lerr.max() <= LSE_MAX, (what, lerr.max())
+    return err.max(), err.mean(), lerr.max()
+
+
+def check_case(moba, dev, B, N, Hq, Hkv, bs, topk, seed, rows=None):
+    host, (q, k, v) = _inputs(B, N, Hq, Hkv, bs, seed, dev)
+    if rows is None:
+        rows = oracle.all_rows(B, Hq, N)
+    kbar = oracle.pool(host[1], bs)
+    sel, s_last, s_next = oracle.select(host[0], kbar, Hkv, bs, topk, rows)
+    ref_out, ref_lse = oracle.attend(*host, bs, topk, rows, sel)
+
+    idx = moba.gate(q, k, bs, topk)
+    out, lse = moba.forward(q, k, v, bs, topk)
+    assert moba.sync_status() == 0
+    gidx = idx.cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
+
+    tie = oracle.near_tie(s_last, s_next)
+    mism = (gidx != sel).any(axis=1)
+    assert not (mism & ~tie).any(), f"{(mism & ~tie).sum()} selection mismatches outside near ties"
+    go, gl = _gather(out, lse, rows)
+    ok = ~mism
+    _compare_outputs(go[ok], gl[ok], ref_out[ok], ref_lse[ok], "forward")
+    if mism.any():  # re-check the near-tie rows with the oracle's selection injected
+        full = idx.clone()
+        full[rows[mism, 0], rows[mism, 1], rows[mism, 2]] = torch.from_numpy(sel[mism]).to(dev)
+        o2, l2 = moba.forward_selected(q, k, v, full, bs, topk)
+        assert moba.sync_status() == 0
+        go2, gl2 = _gather(o2, l2, rows)
+        _compare_outputs(go2[mism], gl2[mism], ref_out[mism], ref_lse[mism], "injected")
+    return {"rows": len(rows), "near_ties": int(tie.sum()), "mismatches": int(mism.sum())}
+
+
+SMALL = [  # B, N, Hq, Hkv, block_size, topk
+    (1, 4096, 1, 1, 512, 3),      # the tiny reference configuration (seed 0)
+    (2, 1000, 4, 2, 128, 3),      # ragged last block, GQA 2
+    (1, 777, 2, 1, 64, 1),        # only the own block
+    (1, 600, 2, 2, 128, 8),       # topk > number of blocks: dense causal
+    (1, 1500, 2, 2, 200, 4),      # block size not a multiple of 128
+    (1, 1024, 8, 1, 128, 3),      # GQA group 8
+    (1, 1, 1, 1, 128, 3),         # one token
+    (1, 130, 1, 1, 128, 2),       # two tiles, one row in the second
+    (2, 2048, 4, 4, 256, 5),
+]
+
+
+@pytest.mark.parametrize("case", SMALL)
+def test_small_cases_all_rows(moba, cuda_dev, case):
+    B, N, Hq, Hkv, bs, topk = case
+    seed = 0 if case == SMALL[0] else 100 + SMALL.index(case)
+    check_case(moba, cuda_dev, B, N, Hq, Hkv, bs, topk, seed)
+
+
+def test_single_head_long_sequence(moba, cuda_dev):
+    """Single head, N=32768, block 2048, top-3 (seed 1); sampled rows for the outputs."""
+    B, N, Hq, Hkv, bs, topk = 1, 32768, 1, 1, 2048, 3
+    check_case(moba, cuda_dev, B, N, Hq, Hkv, bs, topk, 1, rows=sample_rows(B, Hq, N, bs, topk, 2048))
+
+
+def test_fine_granularity_gqa(moba, cuda_dev):
+    """B=2, Hq=32, Hkv=8, N=32768, block 256, top-32 (seed 2); sampled rows."""
+    B, N, Hq, Hkv, bs, topk = 2, 32768, 32, 8, 256, 32
+    check_case(moba, cuda_dev, B, N, Hq, Hkv, bs, topk, 2, rows=sample_rows(B, Hq, N, bs, topk, 48))
+
+
+def test_dense_causal_matches_oracle(moba, cuda_dev):
+    B, N, Hq, Hkv = 1, 700, 4, 2
+    host, (q, k, v) = _inputs(B, N, Hq, Hkv, 128, 7, cuda_dev)
+    rows = oracle.all_rows(B, Hq, N)
+    nblk = (N + 127) // 128
+    r = oracle.forward(*host, 128, nblk, rows)
+    out, lse = moba.dense_causal(q, k, v)
+    assert moba.sync_status() == 0
+    go, gl = _gather(out, lse, rows)
+    _compare_outputs(go, gl, r["out"], r["lse"], "dense")
+
+
+def test_forward_is_deterministic(moba, cuda_dev):
+    _, (q, k, v) = _inputs(1, 3000, 4, 2, 256, 5, cuda_dev)
+    o1, l1 = moba.forward(q, k, v, 256, 4)
+    o2, l2 = moba.forward(q, k, v, 256, 4)
+    assert moba.sync_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_malformed_selection_sets_error_flag(moba, cuda_dev):
+    B, N, Hq, Hkv, bs, topk = 1, 512, 1, 1, 128, 2
+    _, (q, k, v) = _inputs(B, N, Hq, Hkv, bs, 3, cuda_dev)
+    idx = moba.gate(q, k, bs, topk)
+    good_out, good_lse = moba.forward_selected(q, k, v, idx, bs, topk)
+    assert moba.sync_status() == 0
+    bad = idx.clone()
+    bad[0, 0, 200] = torch.tensor([3, 1], dtype=torch.int32)  # a future block, and not ascending
+    out, lse = moba.forward_selected(q, k, v, bad, bs, topk)
+    assert moba.sync_status() == 9  # MOBA_ERR_SELECTION
+    assert torch.isnan(lse[0, 0, 200])
+    keep = torch.ones(N, dtype=torch.bool)
+    keep[200] = False
+    assert torch.equal(lse[0, 0, keep], good_lse[0, 0, keep])
+    assert moba.sync_status() == 0  # the flag was cleared
