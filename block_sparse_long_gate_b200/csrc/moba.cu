@@ -23,7 +23,7 @@
 
 namespace {
 
-int g_attn_impl = 1;  // 0 tensor cores, 1 CUDA cores
+int g_attn_impl = 0;  // 0 tensor cores, 1 CUDA cores
 int g_gate_impl = 0;
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -40,6 +40,7 @@ int make_plan(int B, int Hq, int Hkv, int64_t N, int d, int bs, int topk, Plan* 
     if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || bs < 1 || topk < 1) return MOBA_ERR_SHAPE;
     if (d != MOBA_D || Hq % Hkv != 0 || topk > MOBA_MAX_TOPK || N >= ((int64_t)1 << 31)) return MOBA_ERR_SHAPE;
     if (B > 65535 || Hq > 65535) return MOBA_ERR_SHAPE;
+    if ((int64_t)B * N >= ((int64_t)1 << 31)) return MOBA_ERR_SHAPE;  // TMA row coordinates are 32-bit
     Plan& P = *p;
     P.B = B;
     P.Hq = Hq;

@@ -33,7 +33,7 @@
  *   - Asynchronous failures (a kernel wait that hit its iteration limit, a
  *     launch error) are reported by moba_sync_status().
  *   - Supported: d = 128, Hq % Hkv == 0, 1 <= topk <= 64, block_size >= 1,
- *     1 <= N < 2^31, ceil(N / block_size) <= 16384, B and Hq <= 65535, and a
+ *     1 <= N, B * N < 2^31, ceil(N / block_size) <= 16384, B and Hq <= 65535, and a
  *     device of compute capability 10.0 (sm_100a).
  */
 #ifndef MOBA_H
