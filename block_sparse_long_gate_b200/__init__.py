@@ -30,8 +30,10 @@ STATUS_NAMES = {
 EXPORTED = [
     "moba_status_string", "moba_workspace_size", "moba_forward", "moba_forward_ws", "moba_gate",
     "moba_forward_selected", "moba_forward_selected_ws", "moba_dense_causal", "moba_sync_status",
-    "moba_set_attention_impl", "moba_set_gate_impl",
+    "moba_set_attention_impl", "moba_set_gate_impl", "moba_stage_timing", "moba_stage_times",
+    "moba_launch_count",
 ]
+STAGES = ("pool", "gate", "invert", "attention", "merge")
 
 
 class MobaError(RuntimeError):
@@ -80,6 +82,12 @@ def lib():
             L.moba_set_attention_impl.argtypes = [_I]
             L.moba_set_gate_impl.restype = _I
             L.moba_set_gate_impl.argtypes = [_I]
+            L.moba_stage_timing.restype = _I
+            L.moba_stage_timing.argtypes = [_I]
+            L.moba_stage_times.restype = _I
+            L.moba_stage_times.argtypes = [ctypes.POINTER(ctypes.c_float), _I, ctypes.POINTER(ctypes.c_int)]
+            L.moba_launch_count.restype = ctypes.c_uint64
+            L.moba_launch_count.argtypes = []
             _lib = L
     return _lib
 
@@ -189,3 +197,21 @@ def set_attention_impl(impl: int) -> int:
 
 def set_gate_impl(impl: int) -> int:
     return int(lib().moba_set_gate_impl(impl))
+
+
+def stage_timing(enable: bool) -> bool:
+    """Record CUDA events between the stages of every forward call (for measurement)."""
+    return bool(lib().moba_stage_timing(1 if enable else 0))
+
+
+def stage_times() -> tuple[dict, int]:
+    """({stage: ms summed over the recorded calls}, number of calls); clears the records."""
+    arr = (ctypes.c_float * len(STAGES))()
+    calls = ctypes.c_int(0)
+    _check(lib().moba_stage_times(arr, len(STAGES), ctypes.byref(calls)), "moba_stage_times")
+    return {name: float(arr[i]) for i, name in enumerate(STAGES)}, int(calls.value)
+
+
+def launch_count() -> int:
+    """Kernels launched by libmoba so far in this process."""
+    return int(lib().moba_launch_count())

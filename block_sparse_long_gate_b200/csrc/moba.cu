@@ -12,6 +12,10 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <atomic>
+#include <mutex>
+#include <vector>
+
 #include "common.cuh"
 #include "k_attn_common.cuh"
 #include "k_attn_simt.cuh"
@@ -25,6 +29,44 @@ namespace {
 
 int g_attn_impl = 0;  // 0 tensor cores, 1 CUDA cores
 int g_gate_impl = 0;
+
+// Kernel launches made by the library (all devices, all threads).
+std::atomic<uint64_t> g_launches{0};
+
+// Optional per-stage timing: CUDA events recorded between the stages of each
+// forward call, on the call's stream.
+constexpr int kStages = 5;  // pool, gate, invert, attention, merge
+struct StageRec {
+    cudaEvent_t ev[kStages + 1];
+};
+std::mutex g_timing_mu;
+bool g_timing = false;
+std::vector<StageRec> g_recs;
+
+struct StageTimer {
+    StageRec rec;
+    bool on = false;
+    cudaStream_t st;
+    explicit StageTimer(cudaStream_t s) : st(s) {
+        std::lock_guard<std::mutex> lk(g_timing_mu);
+        if (!g_timing) return;
+        on = true;
+        for (int i = 0; i <= kStages; ++i)
+            if (cudaEventCreate(&rec.ev[i]) != cudaSuccess) on = false;
+        if (on) cudaEventRecord(rec.ev[0], st);
+    }
+    void mark(int stage) {  // end of stage `stage` (0-based)
+        if (on) cudaEventRecord(rec.ev[stage + 1], st);
+    }
+    void finish(int upto) {
+        if (!on) return;
+        for (int i = upto; i < kStages; ++i) cudaEventRecord(rec.ev[i + 1], st);
+        std::lock_guard<std::mutex> lk(g_timing_mu);
+        g_recs.push_back(rec);
+    }
+};
+
+inline void count_launch(int n = 1) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -123,6 +165,7 @@ int run_pool(const Plan& P, const void* k, double* kbar, cudaStream_t st) {
     if (P.nfull == 0) return MOBA_OK;
     dim3 grid((unsigned)P.nfull, P.Hkv, P.B);
     moba_pool_kernel<<<grid, POOL_THREADS, 0, st>>>((const uint16_t*)k, kbar, P.N, P.Hkv, P.bs, P.nfull);
+    count_launch();
     return launch_ok();
 }
 
@@ -137,6 +180,7 @@ int run_gate(const Plan& P, const void* q, const double* kbar, int32_t* idx, cud
         moba_gate_simt_kernel<32><<<grid, GATE_ROWS, 0, st>>>(qq, kbar, idx, P.N, P.Hq, P.Hkv, P.bs, P.topk, P.nfull);
     else
         moba_gate_simt_kernel<64><<<grid, GATE_ROWS, 0, st>>>(qq, kbar, idx, P.N, P.Hq, P.Hkv, P.bs, P.topk, P.nfull);
+    count_launch();
     return launch_ok();
 }
 
@@ -145,6 +189,7 @@ int run_scan(ScanSrc src, int64_t n, int64_t* parts, int64_t* out, cudaStream_t 
     moba_scan_partial_kernel<<<(unsigned)nb, SCAN_THREADS, 0, st>>>(src, n, parts);
     moba_scan_top_kernel<<<1, SCAN_THREADS, 0, st>>>(parts, nb);
     moba_scan_final_kernel<<<(unsigned)nb, SCAN_THREADS, 0, st>>>(src, n, parts, out);
+    count_launch(3);
     return launch_ok();
 }
 
@@ -164,6 +209,7 @@ int run_invert(const Plan& P, const int32_t* idx, char* ws, cudaStream_t st) {
         return MOBA_ERR_CUDA;
     moba_count_kernel<<<grid, INV_THREADS, sm_count, st>>>(idx, counts, P.N, P.Hq, P.Hkv, P.bs, P.topk, P.nblk,
                                                            P.nch);
+    count_launch();
     int rc = launch_ok();
     if (rc) return rc;
     ScanSrc s1{counts, nullptr, 0};
@@ -172,6 +218,7 @@ int run_invert(const Plan& P, const int32_t* idx, char* ws, cudaStream_t st) {
     if ((rc = run_scan(s2, P.L, parts, tiles, st))) return rc;
     moba_scatter_kernel<<<grid, INV_THREADS, sm_scatter, st>>>(idx, segoff, entries, P.N, P.Hq, P.Hkv, P.bs,
                                                                P.topk, P.nblk, P.nch);
+    count_launch();
     return launch_ok();
 }
 
@@ -215,10 +262,13 @@ int run_attention(const Plan& P, const AttnParams& a, cudaStream_t st) {
         for (int64_t i0 = 0; i0 < items; i0 += (int64_t)1 << 30) {
             int64_t n = items - i0 < ((int64_t)1 << 30) ? items - i0 : ((int64_t)1 << 30);
             moba_attn_simt_kernel<<<(unsigned)n, 128, 0, st>>>(a, i0);
+            count_launch();
         }
         return launch_ok();
     }
-    return run_attention_tc(a, st);
+    const int rc = run_attention_tc(a, st);
+    if (rc == MOBA_OK && items > 0) count_launch();
+    return rc;
 }
 
 int run_merge(const Plan& P, const int32_t* idx, char* ws, void* out, float* lse, cudaStream_t st) {
@@ -226,6 +276,7 @@ int run_merge(const Plan& P, const int32_t* idx, char* ws, void* out, float* lse
     moba_merge_kernel<<<(unsigned)cdiv(nrows, 8), 256, 0, st>>>(
         idx, (const uint16_t*)(ws + P.off_opart), (const float*)(ws + P.off_lpart), (uint16_t*)out, lse, P.N, P.Hq,
         P.bs, P.topk, nrows);
+    count_launch();
     return launch_ok();
 }
 
@@ -250,18 +301,29 @@ int forward_impl(const void* q, const void* k, const void* v, const int32_t* idx
         return MOBA_ERR_WORKSPACE;
     }
     const int32_t* idx = idx_in;
+    StageTimer timer(st);
+    int done = 0;
     do {
         if (!idx) {
             int32_t* widx = (int32_t*)(ws + P.off_idx);
             if ((rc = run_pool(P, k, (double*)(ws + P.off_kbar), st))) break;
+            timer.mark(done++);
             if ((rc = run_gate(P, q, (const double*)(ws + P.off_kbar), widx, st))) break;
+            timer.mark(done++);
             idx = widx;
+        } else {
+            timer.mark(done++);
+            timer.mark(done++);
         }
         if ((rc = run_invert(P, idx, ws, st))) break;
+        timer.mark(done++);
         AttnParams a = attn_params(P, q, k, v, out, lse, ws);
         if ((rc = run_attention(P, a, st))) break;
+        timer.mark(done++);
         if ((rc = run_merge(P, idx, ws, out, lse, st))) break;
+        timer.mark(done++);
     } while (0);
+    timer.finish(done);
     if (own) cudaFreeAsync(ws, st);
     return rc;
 }
@@ -374,6 +436,37 @@ int moba_sync_status(moba_stream_t stream) {
     }
     return flag;
 }
+
+int moba_stage_timing(int enable) {
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    int old = g_timing ? 1 : 0;
+    g_timing = enable != 0;
+    return old;
+}
+
+int moba_stage_times(float* ms, int n, int* calls) {
+    if (!ms || n < 1) return MOBA_ERR_NULL;
+    std::vector<StageRec> recs;
+    {
+        std::lock_guard<std::mutex> lk(g_timing_mu);
+        recs.swap(g_recs);
+    }
+    for (int i = 0; i < n; ++i) ms[i] = 0.f;
+    int rc = MOBA_OK;
+    for (auto& r : recs) {
+        if (cudaEventSynchronize(r.ev[kStages]) != cudaSuccess) rc = MOBA_ERR_CUDA;
+        for (int i = 0; i < kStages && i < n; ++i) {
+            float t = 0.f;
+            if (rc == MOBA_OK && cudaEventElapsedTime(&t, r.ev[i], r.ev[i + 1]) == cudaSuccess) ms[i] += t;
+        }
+        for (int i = 0; i <= kStages; ++i) cudaEventDestroy(r.ev[i]);
+    }
+    if (calls) *calls = (int)recs.size();
+    if (rc != MOBA_OK) cudaGetLastError();
+    return rc;
+}
+
+uint64_t moba_launch_count(void) { return g_launches.load(); }
 
 int moba_set_attention_impl(int impl) {
     int old = g_attn_impl;

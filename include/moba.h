@@ -129,6 +129,24 @@ int moba_dense_causal(const void* q, const void* k, const void* v, void* out, fl
  */
 int moba_sync_status(moba_stream_t stream);
 
+/*
+ * Stage timing for measurement. While enabled, every moba_forward* call records
+ * CUDA events on its stream between its stages (0 pool, 1 gate, 2 selection
+ * inversion, 3 attention, 4 merge; the first two are empty when the selection is
+ * given). Returns the previous setting.
+ */
+int moba_stage_timing(int enable);
+
+/*
+ * Waits for the recorded calls, writes the milliseconds of each stage summed over
+ * them into ms[0..n) (n <= 5 used), the number of calls into *calls (may be NULL),
+ * and forgets the records.
+ */
+int moba_stage_times(float* ms, int n, int* calls);
+
+/* Number of kernels the library has launched in this process (all devices). */
+uint64_t moba_launch_count(void);
+
 /* Implementation selector for the attention step: 0 = tensor-core kernel (default),
  * 1 = the simple CUDA-core kernel kept as a cross-check. Returns the previous value. */
 int moba_set_attention_impl(int impl);
