@@ -481,3 +481,4 @@ int moba_set_gate_impl(int impl) {
 }
 
 }  // extern "C"
+
