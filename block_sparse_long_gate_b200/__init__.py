@@ -31,7 +31,7 @@ EXPORTED = [
     "moba_status_string", "moba_workspace_size", "moba_forward", "moba_forward_ws", "moba_gate",
     "moba_forward_selected", "moba_forward_selected_ws", "moba_dense_causal", "moba_sync_status",
     "moba_set_attention_impl", "moba_set_gate_impl", "moba_stage_timing", "moba_stage_times",
-    "moba_launch_count",
+    "moba_launch_count", "moba_gate_noalloc",
 ]
 STAGES = ("pool", "gate", "invert", "attention", "merge")
 
@@ -88,6 +88,8 @@ def lib():
             L.moba_stage_times.argtypes = [ctypes.POINTER(ctypes.c_float), _I, ctypes.POINTER(ctypes.c_int)]
             L.moba_launch_count.restype = ctypes.c_uint64
             L.moba_launch_count.argtypes = []
+            L.moba_gate_noalloc.restype = _I
+            L.moba_gate_noalloc.argtypes = [_P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P]
             _lib = L
     return _lib
 
@@ -153,6 +155,18 @@ def gate(q, k, block_size: int, topk: int, idx=None, stream=None):
     idx = torch.empty((B, Hq, N, topk), dtype=torch.int32, device=q.device) if idx is None else idx
     _check(lib().moba_gate(_ptr(q), _ptr(k), _ptr(idx), B, Hq, Hkv, N, d, block_size, topk, _stream(stream)),
            "moba_gate")
+    return idx
+
+
+def gate_noalloc(q, k, block_size: int, topk: int, idx=None, stream=None):
+    """gate() for callers that cannot allocate device memory during the call: the block means
+    live in a fixed 8 MiB array inside the library (B * Hkv * floor(N / block_size) <= 8192).
+    Calls that overlap on the GPU race on that array. (The output tensor, when not given, is
+    still allocated here by PyTorch; pass `idx` to avoid that too.)"""
+    B, N, Hq, Hkv, d = _check_qkv(q, k)
+    idx = torch.empty((B, Hq, N, topk), dtype=torch.int32, device=q.device) if idx is None else idx
+    _check(lib().moba_gate_noalloc(_ptr(q), _ptr(k), _ptr(idx), B, Hq, Hkv, N, d, block_size, topk,
+                                   _stream(stream)), "moba_gate_noalloc")
     return idx
 
 

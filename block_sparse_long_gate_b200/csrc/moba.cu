@@ -482,3 +482,58 @@ int moba_set_gate_impl(int impl) {
 
 }  // extern "C"
 
+// ---------------------------------------------------------------- allocation-free gate
+// Some callers cannot allocate device memory while they run: serving engines
+// that reserve nearly all HBM up front for their KV cache and hand out only
+// pre-planned buffers (a cudaMallocAsync there either fails or breaks the plan),
+// and embedders with a fixed, audited memory budget that forbids allocation
+// inside a call. moba_gate_noalloc serves them: it runs the same pooling and gate
+// kernels as moba_gate, but the gate's only scratch, the fp64 block means, lives
+// in the fixed array below instead of a stream-ordered allocation.
+//
+// The array is part of the library image: every GPU that loads the library holds
+// its 8 MiB until the process exits. In host code its name is only a host-side
+// stand-in, so the device address is looked up with cudaGetSymbolAddress, once
+// per device, on the first call made with that device current (that first call
+// should therefore come before any stream capture). All calls share the array
+// and it keeps the last call's contents; the pooling kernel overwrites every
+// entry the gate reads, so nothing needs clearing. Calls that overlap on the GPU
+// (different streams, or different host threads, on the same device) race on it.
+#define MOBA_NOALLOC_KBAR_ROWS 8192  // B * Hkv * floor(N / block_size) <= 8192 (8 MiB of doubles)
+static __device__ __align__(256) double g_noalloc_kbar[MOBA_NOALLOC_KBAR_ROWS * MOBA_D];
+
+namespace {
+std::mutex g_noalloc_mu;
+constexpr int kNoallocMaxDevices = 64;
+double* g_noalloc_dev_ptr[kNoallocMaxDevices] = {};
+}  // namespace
+
+extern "C" int moba_gate_noalloc(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv, int64_t N,
+                                 int d, int block_size, int topk, moba_stream_t stream) {
+    Plan P;
+    int rc = make_plan(B, Hq, Hkv, N, d, block_size, topk, &P);
+    if (rc) return rc;
+    if ((int64_t)B * Hkv * P.nfull > MOBA_NOALLOC_KBAR_ROWS) return MOBA_ERR_SHAPE;
+    if ((rc = check_ptrs({q, k, (const void*)idx}))) return rc;
+    if ((rc = check_device())) return rc;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOBA_ERR_CUDA;
+    if (dev < 0 || dev >= kNoallocMaxDevices) return MOBA_ERR_UNSUPPORTED;
+    double* kbar = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (!g_noalloc_dev_ptr[dev]) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_kbar) != cudaSuccess || !p) {
+                cudaGetLastError();
+                return MOBA_ERR_CUDA;
+            }
+            g_noalloc_dev_ptr[dev] = (double*)p;
+        }
+        kbar = g_noalloc_dev_ptr[dev];
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    rc = run_pool(P, k, kbar, st);
+    if (!rc) rc = run_gate(P, q, kbar, idx, st);
+    return rc;
+}

@@ -144,6 +144,22 @@ int moba_stage_timing(int enable);
  */
 int moba_stage_times(float* ms, int n, int* calls);
 
+/*
+ * moba_gate without any device allocation, for callers that cannot allocate
+ * while they run (serving engines that pre-plan every byte of HBM for their KV
+ * cache, embedders with a fixed memory budget). The MoBA pages have no
+ * counterpart: this is a library convenience. Same arguments, results and
+ * kernels as moba_gate; its scratch (the block means) is a fixed 8 MiB device
+ * array inside the library, held by every GPU that loads it until exit.
+ *   - Limit: B * Hkv * floor(N / block_size) <= 8192, else MOBA_ERR_SHAPE.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current; make that first call before any stream capture.
+ *   - All calls share the array: calls that overlap on the GPU race on it.
+ *     Nothing in it needs clearing (each call overwrites what it reads).
+ */
+int moba_gate_noalloc(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv, int64_t N, int d,
+                      int block_size, int topk, moba_stream_t stream);
+
 /* Number of kernels the library has launched in this process (all devices). */
 uint64_t moba_launch_count(void);
 
