@@ -53,6 +53,8 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=("moba", "reference"), default="moba")
     p.add_argument("--seq-len", type=int, default=WORKLOAD["N"], help="override N (diagnostic runs only)")
+    p.add_argument("--hq", type=int, default=None, help="override Hq (diagnostic runs only)")
+    p.add_argument("--hkv", type=int, default=None, help="override Hkv (diagnostic runs only)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -61,11 +63,21 @@ def parse_args(argv=None):
 
 
 # ---------------------------------------------------------------- helpers shared with the tests
-def workload(seq_len: int | None = None) -> dict:
+def workload(seq_len: int | None = None, hq: int | None = None, hkv: int | None = None) -> dict:
     w = dict(WORKLOAD)
     if seq_len:
         w["N"] = int(seq_len)
+    if hq:
+        w["Hq"] = int(hq)
+    if hkv:
+        w["Hkv"] = int(hkv)
     return w
+
+
+def workload_name(w: dict) -> str:
+    if all(w[k] == WORKLOAD[k] for k in ("N", "Hq", "Hkv")):
+        return WORKLOAD_NAME
+    return f"{WORKLOAD_NAME} (diagnostic override: N={w['N']}, Hq={w['Hq']}, Hkv={w['Hkv']})"
 
 
 def useful_flops(w: dict) -> float:
@@ -217,7 +229,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = workload(args.seq_len)
+    w = workload(args.seq_len, args.hq, args.hkv)
     q, k, v = host_inputs(w, w["seed"], pin=False)
     for i in range(args.warmup):
         oracle_sample(q, k, v, w, args.sample_rows, 1000 + i)
@@ -233,7 +245,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD_NAME if w["N"] == WORKLOAD["N"] else f"{WORKLOAD_NAME} (N={w['N']})",
+        "config": {"workload": workload_name(w),
                    "global_batch": w["B"], "seq_len": w["N"], "parallelism": "host cores (OpenMP)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -268,7 +280,7 @@ def run_moba(args):
     import block_sparse_long_gate_b200 as moba
 
     moba.lib()
-    w = workload(args.seq_len)
+    w = workload(args.seq_len, args.hq, args.hkv)
     B, N, Hq, Hkv, d, bs, topk = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], w["block_size"], w["topk"]
     seed = w["seed"] + rank
 
@@ -384,7 +396,7 @@ def run_moba(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD_NAME if N == WORKLOAD["N"] else f"{WORKLOAD_NAME} (N={N})",
+            "config": {"workload": workload_name(w),
                        "global_batch": B * world, "seq_len": N,
                        "parallelism": f"{world} independent forward(s), one per GPU, no collective",
                        "l2": "inputs (12 GiB) far exceed the 126 MB L2; no flush between steps"},

@@ -57,11 +57,81 @@ struct TcBars {
     uint32_t kv_issued[TC_STAGES];  // loads issued per stage (producer bookkeeping)
 };
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Row maximum of 128 fp32 values held as 4 x 32 registers: four independent chains
+// of three-input maxima, so the reduction is throughput- rather than latency-bound.
+__device__ __forceinline__ float row_max128(const uint32_t (&v)[4][32]) {
+    float m[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float a = max3f(__uint_as_float(v[c][0]), __uint_as_float(v[c][1]), __uint_as_float(v[c][2]));
+#pragma unroll
+        for (int j = 3; j + 1 < 32; j += 2) a = max3f(a, __uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1]));
+        m[c] = fmaxf(a, __uint_as_float(v[c][31]));
+    }
+    return max3f(m[0], m[1], fmaxf(m[2], m[3]));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+
+// ---------------------------------------------------------------- packed fp32 pairs
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for a pair of values on the FMA pipe, to take load off the MUFU unit that
+// evaluates ex2.approx (per 128-key step the exponentials would otherwise cost
+// as many cycles as the two MMAs). Method: Cody-Waite style range reduction
+// x = n + f with n = round(x) taken from the low mantissa bits of x + 1.5*2^23,
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial with coefficients fitted here
+// for minimax relative error (7.5e-5, far below the 2^-9 rounding of P to bf16);
+// 2^n is added to the exponent field with an integer add. Inputs are clamped at
+// -126 so the exponent cannot underflow into the sign bit.
+#define EXP2_C0 0x1.fff692p-1f
+#define EXP2_C1 0x1.62f31cp-1f
+#define EXP2_C2 0x1.f0de20p-3f
+#define EXP2_C3 0x1.c3f704p-5f
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+    float x0, x1;
+    f2unpack(x2, x0, x1);
+    x2 = f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const uint64_t t2 = fadd2(x2, f2pack(12582912.f, 12582912.f));       // round(x) in the low bits
+    const uint64_t r2 = fadd2(t2, f2pack(-12582912.f, -12582912.f));     // round(x) as a float
+    const uint64_t fr = ffma2(r2, f2pack(-1.f, -1.f), x2);               // x - round(x)
+    uint64_t p2 = ffma2(f2pack(EXP2_C3, EXP2_C3), fr, f2pack(EXP2_C2, EXP2_C2));
+    p2 = ffma2(p2, fr, f2pack(EXP2_C1, EXP2_C1));
+    p2 = ffma2(p2, fr, f2pack(EXP2_C0, EXP2_C0));
+    float p0, p1, t0, t1;
+    f2unpack(p2, p0, p1);
+    f2unpack(t2, t0, t1);
+    return f2pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                  __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+#define EXP2_POLY_PAIRS 3  // of every 8 pairs of a step, evaluated by exp2_poly2
 
 // Bounded wait that also gives up when another role raised the abort flag.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -276,21 +346,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 const int64_t u0 = ti.klo + (int64_t)i * MOBA_KCHUNK;
                 int64_t lim = ti.khi - 1 - u0;                 // last allowed column by the key range
                 if (tmask - u0 < lim) lim = tmask - u0;        // and by causality
-                float mx = -INFINITY;
-                if (lim >= MOBA_KCHUNK - 1) {
+                if (lim < MOBA_KCHUNK - 1) {
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(sr[c][j]));
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
+                        for (int j = 0; j < 32; ++j)
                             if (c * 32 + j > lim) sr[c][j] = __float_as_uint(-INFINITY);
-                            mx = fmaxf(mx, __uint_as_float(sr[c][j]));
-                        }
                 }
+                const float mx = row_max128(sr);
                 const float m_new = fmaxf(m_used, mx * a.scale_log2);
                 const bool need = m_new > m_used + TC_RESCALE_LOG2;
                 if (__any_sync(0xffffffffu, need)) {
@@ -314,18 +377,49 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 }
                 const float nm = -m_used;
                 uint32_t pk[2][32];
-                float ls = 0.f;
+                if (lim >= MOBA_KCHUNK - 1) {
+                    // unmasked step: exponentials split between the MUFU and the FMA pipe
+                    const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(nm, nm);
+                    uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+                    for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][j]), a.scale_log2, nm));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][j + 1]), a.scale_log2, nm));
-                        const uint32_t w = pack_bf16x2(p0, p1);
-                        ls += p0 + p1;
-                        pk[c >> 1][(c & 1) * 16 + (j >> 1)] = w;
-                    }
-                l += ls;
+                        for (int j = 0; j < 32; j += 2) {
+                            const uint64_t x2 =
+                                ffma2(f2pack(__uint_as_float(sr[c][j]), __uint_as_float(sr[c][j + 1])), sc2, nm2);
+                            uint64_t p2;
+                            if (((j >> 1) & 7) < EXP2_POLY_PAIRS) {
+                                p2 = exp2_poly2(x2);
+                            } else {
+                                float x0, x1;
+                                f2unpack(x2, x0, x1);
+                                p2 = f2pack(ex2_approx(x0), ex2_approx(x1));
+                            }
+                            acc2[(j >> 1) & 3] = fadd2(acc2[(j >> 1) & 3], p2);
+                            float p0, p1;
+                            f2unpack(p2, p0, p1);
+                            pk[c >> 1][(c & 1) * 16 + (j >> 1)] = pack_bf16x2(p0, p1);
+                        }
+                    const uint64_t s2 = fadd2(fadd2(acc2[0], acc2[1]), fadd2(acc2[2], acc2[3]));
+                    float l0, l1;
+                    f2unpack(s2, l0, l1);
+                    l += l0 + l1;
+                } else {
+                    // masked step: MUFU only, so masked keys contribute exactly zero
+                    float ls[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) ls[u] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) {
+                            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][j]), a.scale_log2, nm));
+                            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][j + 1]), a.scale_log2, nm));
+                            pk[c >> 1][(c & 1) * 16 + (j >> 1)] = pack_bf16x2(p0, p1);
+                            ls[(j >> 1) & 7] += p0 + p1;
+                        }
+                    l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+                }
                 tmem_st32(tS, pk[0]);
                 tmem_st32(tS + 32, pk[1]);
                 tc_wait_st();

@@ -11,8 +11,9 @@
 //
 // One thread owns one query row and keeps a sorted list of its best k - 1
 // candidates in registers. Candidates arrive in ascending block order and are
-// inserted only when strictly better than the current last entry, which gives
-// the lowest-index tie-break. Scores are formed with fp64 fused multiply-adds
+// inserted only when strictly better than the current last entry, and the list
+// is ordered by (score desc, block index asc), which gives the lowest-index
+// tie-break. Scores are formed with fp64 fused multiply-adds
 // over exact bf16 query values and the double block means.
 #pragma once
 #include "common.cuh"
@@ -86,7 +87,9 @@ __global__ void __launch_bounds__(GATE_ROWS) moba_gate_simt_kernel(const uint16_
                     int cj = (int)j;
 #pragma unroll
                     for (int i = 0; i < KP; ++i) {
-                        if (cs > ts[i]) {
+                        // order: higher score first, lower block index among equal scores (a block
+                        // pushed down the list may meet an equal score of a higher index)
+                        if (cs > ts[i] || (cs == ts[i] && cj < tj[i])) {
                             double x = ts[i];
                             ts[i] = cs;
                             cs = x;

@@ -1,0 +1,449 @@
+// k_gate_tc.cuh - parameter-less gating and top-k on the sm_100a tensor cores.
+//
+// Same selection as the fp64 gate (k_gate.cuh): for query t in block c, the
+// k - 1 best earlier blocks by <q_t, Kbar_j> (higher first, lower index on equal
+// scores) plus c ("MoBA project hub", Step 2; "MoBA tech-report summary",
+// section 2 gating and causality; "KIMI MoBA" blog, section 3 causal_mask and
+// current_block_force).
+//
+// Scores are formed as s~_j = mu_j * sum(q) + <q, r_j>: the block centre mu_j
+// times the row sum in fp32 plus a tcgen05 contraction of the exact bf16 query
+// tile with the residual r_j = Kbar_j - mu_j held as two bf16 planes (hi, lo),
+// accumulated in fp32 in TMEM. |s~_j - s_j| <= eps, a bound derived from the
+// magnitudes involved (computed per row before the boundary pass). One thread owns one query row and keeps
+// the best k - 1 + GATE_EXTRA candidates by s~. Every candidate whose s~ lies
+// within 2 eps of the (k-1)-th best is re-scored exactly (fp64, the same
+// evaluation as the fp64 gate), which decides the boundary exactly:
+//   - candidates with s~ > T + 2 eps are certainly kept,
+//   - the exact top list needs nothing below T - 2 eps,
+// where T is the (k-1)-th best s~. If the kept list cannot show that nothing
+// below it reaches T - 2 eps, the row is re-scored exactly over all candidates.
+//
+// Roles (192 threads, persistent over 128-token tiles of one query head):
+//   warp 0     TMA: Q tile (3-D map over [d, Hq, B*N]),
+//              residual planes of 64 candidate blocks per step into 2 stages
+//   warp 1     tcgen05.mma issuer: S (128 rows x 64 candidates, fp32) = sum over
+//              the two planes and 8 K-steps of Q x plane^T, into 2 TMEM buffers
+//   warps 2-5  top-k: one thread per row (TMEM lane)
+// Shared memory (~113 KB) and TMEM (128 columns) are sized so that two CTAs
+// share an SM and hide each other's latencies.
+#pragma once
+#include <cuda.h>
+
+#include "k_attn_tc.cuh"
+#include "k_pool.cuh"
+
+#define GATE_TC_THREADS 192
+#define GATE_EXTRA 4
+#define GATE_CAND 64                      // candidate blocks per step (MMA N)
+#define GATE_Q_BYTES 32768
+#define GATE_STAGE_BYTES 32768            // 2 planes x 64 rows x 256 B
+#define GATE_GROUP 16                    // scores staged per TMEM load
+#define GATE_SV_BYTES (GATE_GROUP * 128 * 4)
+#define GATE_TC_SMEM (GATE_Q_BYTES + 2 * GATE_STAGE_BYTES + GATE_SV_BYTES + 1024 + 256)  // 2 CTAs per SM
+
+struct __align__(64) GateMaps {
+    CUtensorMap q;       // (d, Hq, B*N), box (64, 1, 128)
+    CUtensorMap planes;  // (d, B*Hkv*2*nfull), box (64, 64)
+};
+
+struct GateParams {
+    const uint16_t* q;
+    const double* kbar;      // [B*Hkv][nfull][d]
+    const float* mu;         // [B*Hkv][nfull]
+    const unsigned* stats;   // [B*Hkv][2]: max |mu|, max |r| (float bits)
+    int32_t* idx;
+    int64_t N, nfull, tiles_per_head, ntiles;
+    int B, Hq, Hkv, G, bs, topk, kp;
+};
+
+struct GateBars {
+    uint64_t q_full, q_empty;
+    uint64_t c_full[2], c_empty[2];
+    uint64_t s_full[2], s_empty[2];
+    uint64_t final_mma;
+    uint32_t tmem_base;
+    int abort_flag;
+    uint32_t issued_q, issued_c[2];
+};
+
+struct GateTile {
+    int b, hq, hk;
+    int64_t t0, nt;   // tokens [t0, t0 + nt)
+    int64_t ncand;    // candidate blocks [0, ncand) scored by the MMA
+    int nch;          // candidate steps of GATE_CAND
+};
+
+__device__ __forceinline__ GateTile gate_tile(const GateParams& p, int64_t item) {
+    GateTile g;
+    const int64_t bh = item / p.tiles_per_head, m = item % p.tiles_per_head;
+    g.b = (int)(bh / p.Hq);
+    g.hq = (int)(bh % p.Hq);
+    g.hk = g.hq / p.G;
+    g.t0 = m * 128;
+    g.nt = (p.N - g.t0 < 128) ? p.N - g.t0 : 128;
+    const int64_t cmax = (g.t0 + g.nt - 1) / p.bs;  // own block of the last row
+    g.ncand = (p.kp > 0 && cmax > p.kp) ? cmax : 0;  // no row needs scores when cmax <= k - 1
+    g.nch = (int)((g.ncand + GATE_CAND - 1) / GATE_CAND);
+    return g;
+}
+
+// Exact fp64 score of one candidate for the thread's query row, reading the row from
+// the swizzled Q tile in shared memory (same evaluation order as the fp64 gate:
+// features ascending, one fused multiply-add each).
+__device__ __forceinline__ double exact_score(const uint8_t* qrow, int r, const double* kb) {
+    double s = 0.0;
+#pragma unroll 2
+    for (int ch = 0; ch < 16; ++ch) {
+        const uint4 v = *reinterpret_cast<const uint4*>(qrow + (ch >> 3) * 16384 + (((ch & 7) ^ (r & 7)) << 4));
+        const double2 k0 = __ldg(reinterpret_cast<const double2*>(kb + ch * 8));
+        const double2 k1 = __ldg(reinterpret_cast<const double2*>(kb + ch * 8 + 2));
+        const double2 k2 = __ldg(reinterpret_cast<const double2*>(kb + ch * 8 + 4));
+        const double2 k3 = __ldg(reinterpret_cast<const double2*>(kb + ch * 8 + 6));
+        s = fma((double)bf16lo(v.x), k0.x, s);
+        s = fma((double)bf16hi(v.x), k0.y, s);
+        s = fma((double)bf16lo(v.y), k1.x, s);
+        s = fma((double)bf16hi(v.y), k1.y, s);
+        s = fma((double)bf16lo(v.z), k2.x, s);
+        s = fma((double)bf16hi(v.z), k2.y, s);
+        s = fma((double)bf16lo(v.w), k3.x, s);
+        s = fma((double)bf16hi(v.w), k3.y, s);
+    }
+    return s;
+}
+
+#ifdef MOBA_GATE_STATS
+__device__ unsigned long long g_gate_stats[4];  // rows scored, zone re-scores, full re-scores, zone size sum
+#define GATE_STAT(i, v) atomicAdd(&g_gate_stats[i], (unsigned long long)(v))
+#else
+#define GATE_STAT(i, v)
+#endif
+
+template <int KPX>
+__global__ void __launch_bounds__(GATE_TC_THREADS, 2)
+    moba_gate_tc_kernel(const GateParams p, const __grid_constant__ GateMaps maps) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* sQ = smem;                     // 32 KB
+    uint8_t* sC = smem + GATE_Q_BYTES;      // 2 x 32 KB
+    float* sV = (float*)(smem + GATE_Q_BYTES + 2 * GATE_STAGE_BYTES);  // [GATE_GROUP][128] score staging
+    GateBars* bars = (GateBars*)(smem + GATE_Q_BYTES + 2 * GATE_STAGE_BYTES + GATE_SV_BYTES);
+    volatile int* abort_flag = &bars->abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->q_full, 1);
+        mbar_init(&bars->q_empty, 1 + 128);  // MMA commit + every top-k thread
+        bars->issued_q = 0;
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->c_full[i], 1);
+            mbar_init(&bars->c_empty[i], 1);
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->s_empty[i], 128);
+            bars->issued_c[i] = 0;
+        }
+        mbar_init(&bars->final_mma, 1);
+        bars->abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, 128);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&maps.q);
+        prefetch_tmap(&maps.planes);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t ti = 0, g = 0;
+            bool ok = true;
+            for (int64_t item = blockIdx.x; item < p.ntiles && ok; item += gridDim.x, ++ti) {
+                const GateTile gt = gate_tile(p, item);
+                // completion #(ti - 1) of q_empty: #(ti - 2) was waited for the previous tile
+                if (!(ok = tc_wait(&bars->q_empty, (ti & 1) ^ 1, abort_flag))) break;
+                mbar_arrive_expect_tx(&bars->q_full, GATE_Q_BYTES);
+                const int row = (int)((int64_t)gt.b * p.N + gt.t0);
+                tma_load_3d(smem_u32(sQ), &maps.q, &bars->q_full, 0, gt.hq, row);
+                tma_load_3d(smem_u32(sQ + 16384), &maps.q, &bars->q_full, 64, gt.hq, row);
+                bars->issued_q += 1;
+                const int64_t bh = (int64_t)gt.b * p.Hkv + gt.hk;
+                for (int m = 0; m < gt.nch; ++m, ++g) {
+                    const uint32_t s = g & 1;
+                    if (!(ok = tc_wait(&bars->c_empty[s], ((g >> 1) & 1) ^ 1, abort_flag))) break;
+                    uint8_t* st = sC + s * GATE_STAGE_BYTES;
+                    mbar_arrive_expect_tx(&bars->c_full[s], GATE_STAGE_BYTES);
+#pragma unroll
+                    for (int pl = 0; pl < 2; ++pl) {
+                        const int r = (int)((bh * 2 + pl) * p.nfull + (int64_t)m * GATE_CAND);
+                        tma_load_3d(smem_u32(st + pl * 16384), &maps.planes, &bars->c_full[s], 0, 0, r);
+                        tma_load_3d(smem_u32(st + pl * 16384 + 8192), &maps.planes, &bars->c_full[s], 64, 0, r);
+                    }
+                    bars->issued_c[s] += 1;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc_bf16(128, GATE_CAND, 0, 0);
+            uint32_t ti = 0, g = 0;
+            bool ok = true;
+            for (int64_t item = blockIdx.x; item < p.ntiles && ok; item += gridDim.x, ++ti) {
+                const GateTile gt = gate_tile(p, item);
+                if (!(ok = tc_wait(&bars->q_full, ti & 1, abort_flag))) break;
+                tc_fence_after();
+                const uint32_t sq = smem_u32(sQ);
+                for (int m = 0; m < gt.nch; ++m, ++g) {
+                    const uint32_t s = g & 1;
+                    if (!(ok = tc_wait(&bars->c_full[s], (g >> 1) & 1, abort_flag))) break;
+                    // the top-k threads have read this TMEM buffer two steps ago
+                    if (!(ok = tc_wait(&bars->s_empty[s], ((g >> 1) & 1) ^ 1, abort_flag))) break;
+                    tc_fence_after();
+                    const uint32_t sc = smem_u32(sC + s * GATE_STAGE_BYTES);
+                    const uint32_t tS = tmem + s * GATE_CAND;
+#pragma unroll
+                    for (int pl = 0; pl < 2; ++pl)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const uint32_t qoff = (k >> 2) * 16384 + (k & 3) * 32;
+                            const uint32_t coff = pl * 16384 + (k >> 2) * 8192 + (k & 3) * 32;
+                            tc_mma_ss(tS, make_sdesc_sw128(sq + qoff, 16, 1024),
+                                      make_sdesc_sw128(sc + coff, 16, 1024), idesc, (pl > 0 || k > 0) ? 1u : 0u);
+                        }
+                    tc_commit(&bars->c_empty[s]);
+                    tc_commit(&bars->s_full[s]);
+                }
+                if (!ok) break;
+                tc_commit(&bars->q_empty);  // the Q tile is no longer read by MMAs
+            }
+            tc_commit(&bars->final_mma);
+            mbar_wait(&bars->final_mma, 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ top-k threads
+        const int r = 32 * (warp & 3) + lane;
+        const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+        const int kp = p.kp;
+        uint32_t ti = 0, g = 0;
+        for (int64_t item = blockIdx.x; item < p.ntiles; item += gridDim.x, ++ti) {
+            const GateTile gt = gate_tile(p, item);
+            if (!tc_wait_warp(&bars->q_full, ti & 1, abort_flag)) break;
+            const bool active = r < gt.nt;
+            const int64_t t = gt.t0 + r;
+            const int64_t c = active ? t / p.bs : 0;
+            const bool need = active && kp > 0 && c > kp;
+            const int64_t bh = (int64_t)gt.b * p.Hkv + gt.hk;
+            const uint8_t* qrow = sQ + r * 128;  // this row of the swizzled tile
+            // row sum and l1 norm (exact in fp64)
+            double sq64 = 0.0, l1 = 0.0;
+#pragma unroll
+            for (int ch = 0; ch < 16; ++ch) {
+                const uint4 v = *reinterpret_cast<const uint4*>(qrow + (ch >> 3) * 16384 + (((ch & 7) ^ (r & 7)) << 4));
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const double a0 = (double)bf16lo(w4[u]), a1 = (double)bf16hi(w4[u]);
+                    sq64 += a0 + a1;
+                    l1 += fabs(a0) + fabs(a1);
+                }
+            }
+            const float sq = (float)sq64;
+            float ts[KPX];
+            int tj[KPX];
+#pragma unroll
+            for (int i = 0; i < KPX; ++i) {
+                ts[i] = -INFINITY;
+                tj[i] = 0x7FFFFFFF;
+            }
+            float thr = -INFINITY;
+            int filled = 0;
+            float smax = 0.f;
+            const float* mu = p.mu + bh * p.nfull;
+            bool ok = true;
+            for (int m = 0; m < gt.nch; ++m, ++g) {
+                const uint32_t s = g & 1;
+                if (!(ok = tc_wait_warp(&bars->s_full[s], (g >> 1) & 1, abort_flag))) break;
+                tc_fence_after();
+                const int64_t j0 = (int64_t)m * GATE_CAND;
+                const int jend = need ? (int)((c - j0 < GATE_CAND) ? c - j0 : GATE_CAND) : 0;  // candidates j < c
+                float* sv = sV + r;  // this row's staged scores, stride 128 (bank = row)
+#pragma unroll 1
+                for (int cc = 0; cc < GATE_CAND / GATE_GROUP; ++cc) {
+                    uint32_t sr[GATE_GROUP];
+                    tmem_ld16(tmem + s * GATE_CAND + lane_off + cc * GATE_GROUP, sr);
+                    tc_wait_ld();
+                    // unrolled pass: scores and the candidates that beat the current threshold
+                    uint32_t hits = 0;
+#pragma unroll
+                    for (int jj = 0; jj < GATE_GROUP; ++jj) {
+                        const int col = cc * GATE_GROUP + jj;
+                        if (col < jend) {
+                            const float v = fmaf(__ldg(mu + j0 + col), sq, __uint_as_float(sr[jj]));
+                            smax = fmaxf(smax, fabsf(v));
+                            sv[jj * 128] = v;
+                            if (v > thr) hits |= 1u << jj;
+                        }
+                    }
+                    // one insertion chain in the code, entered once per hit in ascending block order
+                    while (hits) {
+                        const int jj = __ffs(hits) - 1;
+                        hits &= hits - 1;
+                        float cs = sv[jj * 128];
+                        if (!(cs > thr)) continue;
+                        int cj = (int)(j0 + cc * GATE_GROUP + jj);
+#pragma unroll
+                        for (int i = 0; i < KPX; ++i) {
+                            if (cs > ts[i] || (cs == ts[i] && cj < tj[i])) {
+                                const float x = ts[i];
+                                ts[i] = cs;
+                                cs = x;
+                                const int y = tj[i];
+                                tj[i] = cj;
+                                cj = y;
+                            }
+                        }
+                        if (++filled >= KPX) thr = ts[KPX - 1];
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&bars->s_empty[s]);
+            }
+            if (!ok) break;
+            if (active) {
+                int32_t* orow = p.idx + (((int64_t)gt.b * p.Hq + gt.hq) * p.N + t) * p.topk;
+                if (!need) {
+                    if (c <= kp) {  // every earlier block is kept
+                        for (int i = 0; i < p.topk; ++i) orow[i] = (i < c) ? i : (i == c ? (int32_t)c : -1);
+                    } else {  // topk == 1: only the own block
+                        orow[0] = (int32_t)c;
+                    }
+                } else {
+                    // error bound of s~ (see the file comment): tensor-core accumulation of the residual
+                    // part and its two-plane representation, plus the fp32 centre product and sum.
+                    const float mu_max = __uint_as_float(p.stats[bh * 2 + 0]);
+                    const float r_max = __uint_as_float(p.stats[bh * 2 + 1]);
+                    const double eps = 0x1p-11 * l1 * (double)r_max +
+                                       0x1p-20 * ((double)mu_max * fabs(sq64) + (double)smax) + 1e-30;
+                    float T = 0.f;
+#pragma unroll
+                    for (int i = 0; i < KPX; ++i)
+                        if (i == kp - 1) T = ts[i];
+                    const double lo_thr = (double)T - 2.0 * eps, hi_thr = (double)T + 2.0 * eps;
+                    const double* kb = p.kbar + bh * p.nfull * MOBA_D;
+                    const bool overflow = (c > KPX) && ((double)ts[KPX - 1] >= lo_thr);
+                    GATE_STAT(0, 1);
+                    GATE_STAT(2, overflow ? 1 : 0);
+                    // kept blocks (local array, filled in any order, sorted at the end)
+                    int outj[KPX];
+                    int nout = 0;
+                    // exact candidates: the band [T - 2 eps, T + 2 eps], or every candidate on overflow
+                    int bj[KPX];
+                    int nb = 0;
+                    if (!overflow) {
+#pragma unroll
+                        for (int i = 0; i < KPX; ++i) {
+                            const bool valid = tj[i] != 0x7FFFFFFF;
+                            if (valid && (double)ts[i] > hi_thr) outj[nout++] = tj[i];  // certainly kept
+                            else if (valid && (double)ts[i] >= lo_thr) bj[nb++] = tj[i];
+                        }
+                    }
+                    const int need_n = kp - nout;
+                    // exact top need_n by (score desc, block index asc), insertion into a short list
+                    double es[KPX];
+                    int ej[KPX];
+                    int ne = 0;
+                    const int64_t n_exact = overflow ? c : nb;
+#pragma unroll 1
+                    for (int64_t z = 0; z < n_exact; ++z) {
+                        const int jz = overflow ? (int)z : bj[z];
+                        const double e = exact_score(qrow, r, kb + (int64_t)jz * MOBA_D);
+                        GATE_STAT(3, 1);
+                        int pos = ne;
+                        while (pos > 0 && (e > es[pos - 1] || (e == es[pos - 1] && jz < ej[pos - 1]))) --pos;
+                        if (pos >= need_n) continue;
+                        const int last = ne < need_n ? ne : need_n - 1;
+                        for (int u = last; u > pos; --u) {
+                            es[u] = es[u - 1];
+                            ej[u] = ej[u - 1];
+                        }
+                        es[pos] = e;
+                        ej[pos] = jz;
+                        if (ne < need_n) ++ne;
+                    }
+                    for (int u = 0; u < ne; ++u) outj[nout++] = ej[u];
+                    // ascending block order
+                    for (int i2 = 1; i2 < nout; ++i2) {
+                        const int v = outj[i2];
+                        int u = i2;
+                        while (u > 0 && outj[u - 1] > v) {
+                            outj[u] = outj[u - 1];
+                            --u;
+                        }
+                        outj[u] = v;
+                    }
+                    for (int i2 = 0; i2 < kp; ++i2) orow[i2] = outj[i2];
+                    orow[kp] = (int32_t)c;
+                }
+            }
+            mbar_arrive(&bars->q_empty);  // this row of the Q tile is no longer read
+        }
+    }
+
+    __syncthreads();
+    if (warp == 0 && lane == 0 && *abort_flag) {
+        if (bars->issued_q) mbar_wait(&bars->q_full, (bars->issued_q - 1) & 1);
+        for (int i = 0; i < 2; ++i)
+            if (bars->issued_c[i]) mbar_wait(&bars->c_full[i], (bars->issued_c[i] - 1) & 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 128);
+}
+
+// ---------------------------------------------------------------- host side
+static bool moba_make_2d_map(CUtensorMap* m, const void* base, int64_t rows) {
+    moba_encode_tiled_fn enc = moba_get_encoder();
+    if (!enc) return false;
+    cuuint64_t gdim[3] = {(cuuint64_t)MOBA_D, 1, (cuuint64_t)rows};
+    cuuint64_t gstr[2] = {(cuuint64_t)MOBA_D * 2, (cuuint64_t)MOBA_D * 2};
+    cuuint32_t box[3] = {64, 1, GATE_CAND};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstr, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KPX>
+static int launch_gate_tc(const GateParams& gp, const GateMaps& maps, int grid, cudaStream_t st) {
+    if (cudaFuncSetAttribute(moba_gate_tc_kernel<KPX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GATE_TC_SMEM) != cudaSuccess)
+        return MOBA_ERR_CUDA;
+    moba_gate_tc_kernel<KPX><<<grid, GATE_TC_THREADS, GATE_TC_SMEM, st>>>(gp, maps);
+    return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA;
+}
+
+static int run_gate_tc(const GateParams& gp, const uint16_t* planes, cudaStream_t st) {
+    GateMaps maps;
+    if (!moba_make_kv_map(&maps.q, gp.q, (int64_t)gp.B * gp.N, gp.Hq)) return MOBA_ERR_CUDA;
+    if (!moba_make_2d_map(&maps.planes, planes, (int64_t)gp.B * gp.Hkv * 2 * gp.nfull)) return MOBA_ERR_CUDA;
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return MOBA_ERR_CUDA;
+    const int grid = (int)(gp.ntiles < 2 * nsm ? gp.ntiles : 2 * nsm);
+    if (gp.kp + GATE_EXTRA <= 8) return launch_gate_tc<8>(gp, maps, grid, st);
+    if (gp.kp + GATE_EXTRA <= 16) return launch_gate_tc<16>(gp, maps, grid, st);
+    if (gp.kp + GATE_EXTRA <= 24) return launch_gate_tc<24>(gp, maps, grid, st);
+    if (gp.kp + GATE_EXTRA <= 40) return launch_gate_tc<40>(gp, maps, grid, st);
+    return launch_gate_tc<72>(gp, maps, grid, st);
+}

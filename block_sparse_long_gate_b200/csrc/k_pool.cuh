@@ -16,10 +16,23 @@
 
 #define POOL_THREADS 256
 
+// Extra outputs for the tensor-core gate (all null when only Kbar is wanted):
+// each block mean is written as a centre mu_j (fp32, the mean over the d
+// features) plus a residual r_j = Kbar_j - mu_j split into two bf16 planes
+// (hi = bf16(r), lo = bf16(r - hi)), so that <q, Kbar_j> = mu_j * sum(q) + <q, r_j>
+// with the cancellation-prone part small. head_stats[(b*Hkv+h)*2 + {0,1}] receive
+// max_j |mu_j| and max_{j,d} |r_jd| (float bits, non-negative, so integer atomicMax
+// orders them) for the gate's error bound.
+struct PoolAux {
+    uint16_t* planes;       // bf16 [B*Hkv][2][nfull][d]
+    float* mu;              // fp32 [B*Hkv][nfull]
+    unsigned* head_stats;   // [B*Hkv][2], zeroed before the launch
+};
+
 // grid (nfull, Hkv, B); 16 row groups x 16 threads that each read 16 bytes.
 __global__ void __launch_bounds__(POOL_THREADS) moba_pool_kernel(const uint16_t* __restrict__ K,
                                                                  double* __restrict__ kbar, int64_t N,
-                                                                 int Hkv, int bs, int64_t nfull) {
+                                                                 int Hkv, int bs, int64_t nfull, PoolAux aux) {
     const int64_t j = blockIdx.x;
     const int h = blockIdx.y, b = blockIdx.z;
     const int c16 = threadIdx.x & 15;
@@ -59,10 +72,43 @@ __global__ void __launch_bounds__(POOL_THREADS) moba_pool_kernel(const uint16_t*
 #pragma unroll
     for (int i = 0; i < 8; ++i) red[rg][c16 * 8 + i] = acc[i];
     __syncthreads();
+    double x = 0.0;
     if (threadIdx.x < MOBA_D) {
         double s = 0.0;
 #pragma unroll
         for (int g = 0; g < 16; ++g) s += red[g][threadIdx.x];
-        kbar[(((int64_t)b * Hkv + h) * nfull + j) * MOBA_D + threadIdx.x] = s / (double)bs;
+        x = s / (double)bs;
+        kbar[(((int64_t)b * Hkv + h) * nfull + j) * MOBA_D + threadIdx.x] = x;
+    }
+    if (aux.planes == nullptr) return;
+    // centre and residual planes (threads 0..127 own one feature each)
+    __shared__ double red2[4];
+    __shared__ float fred[4];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    double sx = x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, o);
+    if (lane == 0 && w < 4) red2[w] = sx;
+    __syncthreads();
+    const float mu = (float)((red2[0] + red2[1] + red2[2] + red2[3]) / (double)MOBA_D);
+    const int64_t bh = (int64_t)b * Hkv + h;
+    float ar = 0.f;
+    if (threadIdx.x < MOBA_D) {
+        const double r = x - (double)mu;
+        const __nv_bfloat16 hi = __float2bfloat16_rn((float)r);
+        const __nv_bfloat16 lo = __float2bfloat16_rn((float)(r - (double)__bfloat162float(hi)));
+        aux.planes[((bh * 2 + 0) * nfull + j) * MOBA_D + threadIdx.x] = __bfloat16_as_ushort(hi);
+        aux.planes[((bh * 2 + 1) * nfull + j) * MOBA_D + threadIdx.x] = __bfloat16_as_ushort(lo);
+        ar = (float)fabs(r) * (1.0f + 1.0f / 1024.0f);  // rounded up: a bound on |r|
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ar = fmaxf(ar, __shfl_xor_sync(0xffffffffu, ar, o));
+    if (lane == 0 && w < 4) fred[w] = ar;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const float rm = fmaxf(fmaxf(fred[0], fred[1]), fmaxf(fred[2], fred[3]));
+        aux.mu[bh * nfull + j] = mu;
+        atomicMax(&aux.head_stats[bh * 2 + 0], __float_as_uint(fabsf(mu)));
+        atomicMax(&aux.head_stats[bh * 2 + 1], __float_as_uint(rm));
     }
 }

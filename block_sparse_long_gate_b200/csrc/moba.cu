@@ -21,6 +21,7 @@
 #include "k_attn_simt.cuh"
 #include "k_attn_tc.cuh"
 #include "k_gate.cuh"
+#include "k_gate_tc.cuh"
 #include "k_invert.cuh"
 #include "k_merge.cuh"
 #include "k_pool.cuh"
@@ -74,7 +75,8 @@ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 struct Plan {
     int B, Hq, Hkv, G, d, bs, topk, kp;
     int64_t N, nblk, nfull, L, nch, E, Pmax, D, mb, ml, per_bh, nseg, nscan_parts;
-    size_t off_kbar, off_idx, off_counts, off_segoff, off_tiles, off_parts, off_entries, off_opart, off_lpart;
+    size_t off_kbar, off_planes, off_mu, off_stats, off_idx, off_counts, off_segoff, off_tiles, off_parts, off_entries,
+        off_opart, off_lpart, gate_bytes;
     size_t total;
 };
 
@@ -116,8 +118,16 @@ int make_plan(int B, int Hq, int Hkv, int64_t N, int d, int bs, int topk, Plan* 
     P.nscan_parts = cdiv(nscan, SCAN_TILE);
 
     size_t o = 0;
+    const size_t nf = (size_t)(P.nfull > 0 ? P.nfull : 1);
     P.off_kbar = o;
-    o = align256(o + sizeof(double) * (size_t)B * Hkv * (P.nfull > 0 ? P.nfull : 1) * MOBA_D);
+    o = align256(o + sizeof(double) * (size_t)B * Hkv * nf * MOBA_D);
+    P.off_planes = o;
+    o = align256(o + sizeof(uint16_t) * (size_t)B * Hkv * 2 * nf * MOBA_D);
+    P.off_mu = o;
+    o = align256(o + sizeof(float) * (size_t)B * Hkv * nf);
+    P.off_stats = o;
+    o = align256(o + sizeof(unsigned) * (size_t)B * Hkv * 2);
+    P.gate_bytes = o;  // the gate's scratch is the workspace's first gate_bytes bytes
     P.off_idx = o;
     o = align256(o + sizeof(int32_t) * (size_t)B * Hq * N * topk);
     P.off_counts = o;
@@ -161,15 +171,63 @@ int check_ptrs(std::initializer_list<const void*> ps) {
 int launch_ok() { return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA; }
 
 // ---------------------------------------------------------------- stages
-int run_pool(const Plan& P, const void* k, double* kbar, cudaStream_t st) {
+// Gate scratch inside a workspace: Kbar (fp64) and, for the tensor-core gate, the centre /
+// residual-plane form of it and the per-head magnitude bounds.
+struct GateScratch {
+    double* kbar;
+    PoolAux aux;  // all null: fp64 gate only
+};
+
+GateScratch gate_scratch(const Plan& P, char* ws, bool tc) {
+    GateScratch g;
+    g.kbar = (double*)(ws + P.off_kbar);
+    g.aux.planes = tc ? (uint16_t*)(ws + P.off_planes) : nullptr;
+    g.aux.mu = tc ? (float*)(ws + P.off_mu) : nullptr;
+    g.aux.head_stats = tc ? (unsigned*)(ws + P.off_stats) : nullptr;
+    return g;
+}
+
+bool use_tc_gate(const Plan& P) { return g_gate_impl == 0 && P.nfull > 0 && P.kp > 0; }
+
+int run_pool(const Plan& P, const void* k, const GateScratch& gs, cudaStream_t st) {
     if (P.nfull == 0) return MOBA_OK;
+    if (gs.aux.head_stats &&
+        cudaMemsetAsync(gs.aux.head_stats, 0, sizeof(unsigned) * 2 * (size_t)P.B * P.Hkv, st) != cudaSuccess)
+        return MOBA_ERR_CUDA;
     dim3 grid((unsigned)P.nfull, P.Hkv, P.B);
-    moba_pool_kernel<<<grid, POOL_THREADS, 0, st>>>((const uint16_t*)k, kbar, P.N, P.Hkv, P.bs, P.nfull);
+    moba_pool_kernel<<<grid, POOL_THREADS, 0, st>>>((const uint16_t*)k, gs.kbar, P.N, P.Hkv, P.bs, P.nfull,
+                                                    gs.aux);
     count_launch();
     return launch_ok();
 }
 
-int run_gate(const Plan& P, const void* q, const double* kbar, int32_t* idx, cudaStream_t st) {
+int run_gate_simt(const Plan& P, const void* q, const double* kbar, int32_t* idx, cudaStream_t st);
+
+int run_gate(const Plan& P, const void* q, const GateScratch& gs, int32_t* idx, cudaStream_t st) {
+    if (!gs.aux.planes) return run_gate_simt(P, q, gs.kbar, idx, st);
+    GateParams gp;
+    gp.q = (const uint16_t*)q;
+    gp.kbar = gs.kbar;
+    gp.mu = gs.aux.mu;
+    gp.stats = gs.aux.head_stats;
+    gp.idx = idx;
+    gp.N = P.N;
+    gp.nfull = P.nfull;
+    gp.tiles_per_head = cdiv(P.N, 128);
+    gp.ntiles = gp.tiles_per_head * P.B * P.Hq;
+    gp.B = P.B;
+    gp.Hq = P.Hq;
+    gp.Hkv = P.Hkv;
+    gp.G = P.G;
+    gp.bs = P.bs;
+    gp.topk = P.topk;
+    gp.kp = P.kp;
+    const int rc = run_gate_tc(gp, gs.aux.planes, st);
+    if (rc == MOBA_OK) count_launch();
+    return rc;
+}
+
+int run_gate_simt(const Plan& P, const void* q, const double* kbar, int32_t* idx, cudaStream_t st) {
     dim3 grid((unsigned)cdiv(P.N, GATE_ROWS), P.Hq, P.B);
     const uint16_t* qq = (const uint16_t*)q;
     if (P.kp <= 8)
@@ -273,7 +331,7 @@ int run_attention(const Plan& P, const AttnParams& a, cudaStream_t st) {
 
 int run_merge(const Plan& P, const int32_t* idx, char* ws, void* out, float* lse, cudaStream_t st) {
     int64_t nrows = (int64_t)P.B * P.Hq * P.N;
-    moba_merge_kernel<<<(unsigned)cdiv(nrows, 8), 256, 0, st>>>(
+    moba_merge_kernel<<<(unsigned)cdiv(nrows, MERGE_THREADS / 16), MERGE_THREADS, 0, st>>>(
         idx, (const uint16_t*)(ws + P.off_opart), (const float*)(ws + P.off_lpart), (uint16_t*)out, lse, P.N, P.Hq,
         P.bs, P.topk, nrows);
     count_launch();
@@ -306,9 +364,10 @@ int forward_impl(const void* q, const void* k, const void* v, const int32_t* idx
     do {
         if (!idx) {
             int32_t* widx = (int32_t*)(ws + P.off_idx);
-            if ((rc = run_pool(P, k, (double*)(ws + P.off_kbar), st))) break;
+            const GateScratch gs = gate_scratch(P, ws, use_tc_gate(P));
+            if ((rc = run_pool(P, k, gs, st))) break;
             timer.mark(done++);
-            if ((rc = run_gate(P, q, (const double*)(ws + P.off_kbar), widx, st))) break;
+            if ((rc = run_gate(P, q, gs, widx, st))) break;
             timer.mark(done++);
             idx = widx;
         } else {
@@ -396,15 +455,15 @@ int moba_gate(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv
     if ((rc = check_ptrs({q, k, (const void*)idx}))) return rc;
     if ((rc = check_device())) return rc;
     cudaStream_t st = (cudaStream_t)stream;
-    double* kbar = nullptr;
-    size_t kb_bytes = sizeof(double) * (size_t)B * Hkv * (P.nfull > 0 ? P.nfull : 1) * MOBA_D;
-    if (cudaMallocAsync((void**)&kbar, kb_bytes, st) != cudaSuccess) {
+    char* scratch = nullptr;
+    if (cudaMallocAsync((void**)&scratch, P.gate_bytes, st) != cudaSuccess) {
         cudaGetLastError();
         return MOBA_ERR_OOM;
     }
-    rc = run_pool(P, k, kbar, st);
-    if (!rc) rc = run_gate(P, q, kbar, idx, st);
-    cudaFreeAsync(kbar, st);
+    const GateScratch gs = gate_scratch(P, scratch, use_tc_gate(P));
+    rc = run_pool(P, k, gs, st);
+    if (!rc) rc = run_gate(P, q, gs, idx, st);
+    cudaFreeAsync(scratch, st);
     return rc;
 }
 
@@ -533,7 +592,21 @@ extern "C" int moba_gate_noalloc(const void* q, const void* k, int32_t* idx, int
         kbar = g_noalloc_dev_ptr[dev];
     }
     cudaStream_t st = (cudaStream_t)stream;
-    rc = run_pool(P, k, kbar, st);
-    if (!rc) rc = run_gate(P, q, kbar, idx, st);
+    GateScratch gs;
+    gs.kbar = kbar;
+    gs.aux = PoolAux{nullptr, nullptr, nullptr};  // the fp64 gate: its only scratch is Kbar
+    rc = run_pool(P, k, gs, st);
+    if (!rc) rc = run_gate(P, q, gs, idx, st);
     return rc;
 }
+
+#ifdef MOBA_GATE_STATS
+extern "C" int moba_debug_gate_stats(unsigned long long* out4, int reset) {
+    if (cudaMemcpyFromSymbol(out4, g_gate_stats, sizeof(unsigned long long) * 4) != cudaSuccess) return MOBA_ERR_CUDA;
+    if (reset) {
+        unsigned long long z[4] = {0, 0, 0, 0};
+        if (cudaMemcpyToSymbol(g_gate_stats, z, sizeof(z)) != cudaSuccess) return MOBA_ERR_CUDA;
+    }
+    return MOBA_OK;
+}
+#endif
