@@ -31,7 +31,7 @@ EXPORTED = [
     "moba_status_string", "moba_workspace_size", "moba_forward", "moba_forward_ws", "moba_gate",
     "moba_forward_selected", "moba_forward_selected_ws", "moba_dense_causal", "moba_sync_status",
     "moba_set_attention_impl", "moba_set_gate_impl", "moba_stage_timing", "moba_stage_times",
-    "moba_launch_count", "moba_gate_noalloc",
+    "moba_launch_count", "moba_gate_noalloc", "moba_last_error_string",
 ]
 STAGES = ("pool", "gate", "invert", "attention", "merge")
 
@@ -39,7 +39,13 @@ STAGES = ("pool", "gate", "invert", "attention", "merge")
 class MobaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({_status_string(status)})")
+        detail = _status_string(status)
+        if status == 5:  # MOBA_ERR_CUDA: add the runtime's own message
+            try:
+                detail += ": " + lib().moba_last_error_string().decode()
+            except Exception:
+                pass
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({detail})")
 
 
 _lock = threading.Lock()
@@ -88,6 +94,8 @@ def lib():
             L.moba_stage_times.argtypes = [ctypes.POINTER(ctypes.c_float), _I, ctypes.POINTER(ctypes.c_int)]
             L.moba_launch_count.restype = ctypes.c_uint64
             L.moba_launch_count.argtypes = []
+            L.moba_last_error_string.restype = ctypes.c_char_p
+            L.moba_last_error_string.argtypes = []
             L.moba_gate_noalloc.restype = _I
             L.moba_gate_noalloc.argtypes = [_P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P]
             _lib = L

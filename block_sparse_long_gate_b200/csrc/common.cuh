@@ -20,6 +20,9 @@ __device__ int g_moba_err;
 
 __device__ __forceinline__ void moba_set_error(int code) { atomicCAS(&g_moba_err, 0, code); }
 
+// Host: remember the text of a CUDA error for moba_last_error_string().
+void moba_note_cuda_error(cudaError_t e);
+
 // Iteration limit of every spin-wait in the library. A wait that reaches it
 // records MOBA_ERR_DEVICE_TIMEOUT and the kernel leaves the wait. With the
 // nanosleep back-off below this is several seconds of waiting.

@@ -11,9 +11,11 @@
 
 __global__ void __launch_bounds__(128) moba_attn_simt_kernel(AttnParams a, int64_t item0) {
     const int64_t item = item0 + blockIdx.x;
-    const TileInfo ti = decode_tile(a, item);
-    if (ti.kind < 0) return;
+    const PairInfo pi = decode_pair(a, item);
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int x = 0; x < 2; ++x) {
+    const TileInfo& ti = pi.t[x];
+    if (ti.kind < 0) continue;
     const int64_t nrows = ti.kind == 0 ? ti.ne : ti.nt;
     for (int64_t r = w; r < nrows; r += 4) {
         int64_t t;
@@ -63,5 +65,6 @@ __global__ void __launch_bounds__(128) moba_attn_simt_kernel(AttnParams a, int64
             *reinterpret_cast<uint2*>(a.out + (((int64_t)ti.b * a.N + t) * a.Hq + hq) * MOBA_D + lane * 4) = ow;
             if (lane == 0) a.lse[((int64_t)ti.b * a.Hq + hq) * a.N + t] = lse;
         }
+    }
     }
 }

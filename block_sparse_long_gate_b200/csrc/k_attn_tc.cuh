@@ -1,25 +1,37 @@
 // k_attn_tc.cuh - block-sparse attention on the sm_100a tensor cores.
 //
-// One 128-row query tile (past-block list tile, own-block tile or dense tile,
-// see k_attn_common.cuh) is attended against its key range in steps of 128
-// keys ("MoBA project hub", Step 3; "NSA vs MoBA" blog, section 1 formula):
-//   S = Q K^T                     tcgen05.mma, A = Q (smem), B = K (smem), D in TMEM
-//   P = exp2(S * log2(e)/sqrt(d) - m)   softmax warps, one thread per TMEM lane (row)
-//   O += P V                      tcgen05.mma, A = P (TMEM, aliased over S), B = V (smem)
+// A work item is a pair of 128-row query tiles A and B that read the same keys
+// (see k_attn_common.cuh), attended in steps of 128 keys ("MoBA project hub",
+// Step 3; "NSA vs MoBA" blog, section 1 formula). For each tile X:
+//   S_X = Q_X K^T                  tcgen05.mma, A = Q_X (smem), B = K (smem), D in TMEM
+//   P_X = exp2(S_X * log2(e)/sqrt(d) - m_X)   softmax warps of X, one thread per TMEM lane
+//   O_X += P_X V                   tcgen05.mma, A = P_X (TMEM, over S_X), B = V (smem)
 // with a running row maximum m and sum l; the result is O / l and
 // lse = (m + log2 l) * ln 2.
 //
-// Roles (192 threads, one CTA per SM, persistent over the work items):
-//   warp 0     producer: TMA loads of the K and V steps into a 3-stage ring
-//   warp 1     MMA issuer (one thread) and TMEM owner
-//   warps 2-5  softmax: gather the tile's Q rows (cp.async), softmax per step,
-//              lazy O rescaling, epilogue (normalise, store bf16 rows + lse)
-// TMEM: S0 = columns [0,128), S1 = [128,256), O = [256,384) (fp32, 128 lanes).
+// Why pairs: one tile's steps form a strict chain (Q K^T -> softmax -> P V ->
+// next Q K^T into the same S). Two tiles interleave on the tensor core - while
+// the softmax warps of A work on S_A, the MMAs of B run - and each K/V step in
+// shared memory feeds twice the MMA work.
+//
+// Roles (320 threads, one CTA per SM, persistent over the pairs):
+//   warp 0     producer: TMA loads of K steps into a 3-slot ring and of V steps
+//              into a 2-slot ring (3-D maps, 128-byte swizzle); K runs one step ahead
+//   warp 1     MMA issuer (one thread) and TMEM owner. Per step i of a pair:
+//              [P V of A for step i-1, Q K^T of A for step i], then the same for B
+//   warps 2-5  softmax of tile A; warps 6-9 softmax of tile B. Each thread owns one
+//              row: gathers its Q row (cp.async, swizzled), runs the softmax with a
+//              lazily moved maximum, and writes the normalised row in the epilogue.
+// TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512) (fp32, 128 lanes).
+// P_X (bf16 pairs) overwrites columns [64,128) of S_X once they have been read.
 // The running maximum used for P only moves when the row maximum grows by more
 // than 2^8 (log2 units), so O is rescaled rarely; P <= 2^8 stays exact in range.
 //
-// Phase rule: a parity wait for completion #k of a barrier is only sound when
-// completion #k-1 is already known to have happened; each wait below names why.
+// Ordering facts the waits rely on:
+//   - the commit after Q K^T of X for step i also covers the P V of X for step
+//     i - 1 issued before it, so "S_X ready" implies O_X holds every step so far;
+//   - a parity wait for completion #k of a barrier is only sound when completion
+//     #k-1 is known to have happened; each wait below says why it holds.
 //
 // Every wait is bounded. A wait that reaches its limit records
 // MOBA_ERR_DEVICE_TIMEOUT and raises a CTA-wide abort flag; all roles then leave
@@ -30,11 +42,12 @@
 
 #include "k_attn_common.cuh"
 
-#define TC_STAGES 3
-#define TC_THREADS 192
-#define TC_STAGE_BYTES 65536  // K step 32 KB + V step 32 KB
+#define TC_THREADS 320
+#define TC_KSLOTS 3
+#define TC_VSLOTS 2
+#define TC_STEP_BYTES 32768  // one K or V step: 128 keys x 128 d x bf16
 #define TC_Q_BYTES 32768
-#define TC_SMEM_BYTES (TC_Q_BYTES + TC_STAGES * TC_STAGE_BYTES + 1024 + 256)
+#define TC_SMEM_BYTES (2 * TC_Q_BYTES + (TC_KSLOTS + TC_VSLOTS) * TC_STEP_BYTES + 512)
 #define TC_RESCALE_LOG2 8.0f
 
 struct __align__(64) TcMaps {
@@ -43,19 +56,21 @@ struct __align__(64) TcMaps {
 };
 
 struct TcBars {
-    uint64_t kv_full[TC_STAGES];
-    uint64_t kv_empty[TC_STAGES];
-    uint64_t q_full;
-    uint64_t s_full[2];
-    uint64_t p_full[2];
-    uint64_t pv_done;  // one completion per step: O holds P V of that step (used by the rescale)
-    uint64_t o_full;   // one completion per tile: the tile's last P V is in O (used by the epilogue)
-    uint64_t o_empty;
+    uint64_t k_full[TC_KSLOTS], k_empty[TC_KSLOTS];
+    uint64_t v_full[TC_VSLOTS], v_empty[TC_VSLOTS];
+    uint64_t q_full[2];   // per tile: its 128 softmax threads gathered their Q rows
+    uint64_t s_full[2];   // per tile: Q K^T of a step is in S_X (and P V of the previous step in O_X)
+    uint64_t p_full[2];   // per tile: P_X of a step is in TMEM
+    uint64_t o_full[2];   // per tile: the tile's last P V is in O_X
+    uint64_t o_empty[2];  // per tile: the epilogue has read O_X
     uint64_t final_mma;
     uint32_t tmem_base;
     int abort_flag;
-    uint32_t kv_issued[TC_STAGES];  // loads issued per stage (producer bookkeeping)
+    uint32_t k_issued[TC_KSLOTS], v_issued[TC_VSLOTS];  // loads issued per slot (teardown bookkeeping)
 };
+
+static_assert(sizeof(TcBars) <= 512, "barrier block does not fit the shared-memory budget");
+static_assert(TC_SMEM_BYTES <= 227 * 1024, "over the per-block shared-memory limit");
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float r;
@@ -75,6 +90,17 @@ __device__ __forceinline__ float row_max128(const uint32_t (&v)[4][32]) {
         m[c] = fmaxf(a, __uint_as_float(v[c][31]));
     }
     return max3f(m[0], m[1], fmaxf(m[2], m[3]));
+}
+
+__device__ __forceinline__ float row_max32(const uint32_t (&v)[32]) {
+    float a0 = max3f(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+    float a1 = max3f(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5]));
+#pragma unroll
+    for (int j = 6; j + 3 < 32; j += 4) {
+        a0 = max3f(a0, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+        a1 = max3f(a1, __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+    }
+    return max3f(a0, a1, fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31])));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -133,8 +159,66 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
 }
 #define EXP2_POLY_PAIRS 3  // of every 8 pairs of a step, evaluated by exp2_poly2
 
+// Masks the columns of a 64-key half (first column index c0) beyond `lim`.
+__device__ __forceinline__ void mask_cols(uint32_t (&sr)[2][32], int c0, int64_t lim) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (c0 + c * 32 + j > lim) sr[c][j] = __float_as_uint(-INFINITY);
+}
+
+// P = exp2(s * scale - m) for 64 keys into 32 bf16 pairs; returns their fp32 sum.
+// `mixed` splits the exponentials between the MUFU and the FMA pipe (only for
+// unmasked keys: the FMA form clamps, the MUFU form gives exact zeros for -inf).
+__device__ __forceinline__ float softmax_half(const uint32_t (&sr)[2][32], uint32_t (&pk)[32], float scale,
+                                              float nm, bool mixed) {
+    float lsum;
+    if (mixed) {
+        const uint64_t sc2 = f2pack(scale, scale), nm2 = f2pack(nm, nm);
+        uint64_t acc2[2] = {0ull, 0ull};
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                const uint64_t x2 = ffma2(f2pack(__uint_as_float(sr[c][j]), __uint_as_float(sr[c][j + 1])), sc2, nm2);
+                uint64_t p2;
+                if (((j >> 1) & 7) < EXP2_POLY_PAIRS) {
+                    p2 = exp2_poly2(x2);
+                } else {
+                    float x0, x1;
+                    f2unpack(x2, x0, x1);
+                    p2 = f2pack(ex2_approx(x0), ex2_approx(x1));
+                }
+                acc2[(j >> 1) & 1] = fadd2(acc2[(j >> 1) & 1], p2);
+                float p0, p1;
+                f2unpack(p2, p0, p1);
+                pk[c * 16 + (j >> 1)] = pack_bf16x2(p0, p1);
+            }
+        float l0, l1;
+        f2unpack(fadd2(acc2[0], acc2[1]), l0, l1);
+        lsum = l0 + l1;
+    } else {
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][j]), scale, nm));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][j + 1]), scale, nm));
+                pk[c * 16 + (j >> 1)] = pack_bf16x2(p0, p1);
+                ls[(j >> 1) & 3] += p0 + p1;
+            }
+        lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+    }
+    return lsum;
+}
+
 // Bounded wait that also gives up when another role raised the abort flag.
-__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// `backoff` adds a short sleep between polls (for roles off the critical path,
+// so their spinning does not take issue slots from the softmax warps).
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                        bool backoff = false) {
     uint32_t n = 0;
     while (!mbar_try_wait(bar, parity)) {
         if (*abort_flag) return false;
@@ -143,7 +227,7 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
             *abort_flag = 1;
             return false;
         }
-        if (n > 64) __nanosleep(64);
+        if (backoff) __nanosleep(128);
     }
     return true;
 }
@@ -154,35 +238,51 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, vol
     return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ int64_t tile_steps(const TileInfo& ti) {
-    return (ti.khi - ti.klo + MOBA_KCHUNK - 1) / MOBA_KCHUNK;
-}
+#ifdef MOBA_ATTN_TRACE
+// Debug timeline of CTA 0 (debug builds only): slot [code][step] = clock64().
+__device__ unsigned long long* g_attn_trace;
+__device__ unsigned int g_attn_trace_n;
+#define ATRACE(code, step)                                                         \
+    do {                                                                           \
+        if (blockIdx.x == 0 && g_attn_trace && (step) < 4096u)                     \
+            g_attn_trace[(unsigned)(code) * 4096u + (unsigned)(step)] = clock64(); \
+    } while (0)
+#else
+#define ATRACE(code, step)
+#endif
 
 __global__ void __launch_bounds__(TC_THREADS, 1)
     moba_attn_tc_kernel(const AttnParams a, const __grid_constant__ TcMaps maps, int64_t items) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t* sQ = smem;
-    uint8_t* sKV = smem + TC_Q_BYTES;
-    TcBars* bars = (TcBars*)(smem + TC_Q_BYTES + TC_STAGES * TC_STAGE_BYTES);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    if (smem_u32(smem_raw) & 1023) {  // the swizzled layout below needs a 1024-byte aligned window
+        if (threadIdx.x == 0) moba_set_error(MOBA_ERR_UNSUPPORTED);
+        return;
+    }
+    uint8_t* sQ = smem_raw;                                  // Q_A, Q_B: 2 x 32 KB
+    uint8_t* sK = smem_raw + 2 * TC_Q_BYTES;                 // K ring
+    uint8_t* sV = sK + TC_KSLOTS * TC_STEP_BYTES;            // V ring
+    TcBars* bars = (TcBars*)(sV + TC_VSLOTS * TC_STEP_BYTES);
     volatile int* abort_flag = &bars->abort_flag;
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < TC_STAGES; ++s) {
-            mbar_init(&bars->kv_full[s], 1);
-            mbar_init(&bars->kv_empty[s], 1);
-            bars->kv_issued[s] = 0;
+        for (int s = 0; s < TC_KSLOTS; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+            bars->k_issued[s] = 0;
         }
-        mbar_init(&bars->q_full, 128);
-        mbar_init(&bars->s_full[0], 1);
-        mbar_init(&bars->s_full[1], 1);
-        mbar_init(&bars->p_full[0], 128);
-        mbar_init(&bars->p_full[1], 128);
-        mbar_init(&bars->pv_done, 1);
-        mbar_init(&bars->o_full, 1);
-        mbar_init(&bars->o_empty, 128);
+        for (int s = 0; s < TC_VSLOTS; ++s) {
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
+            bars->v_issued[s] = 0;
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bars->q_full[x], 128);
+            mbar_init(&bars->s_full[x], 1);
+            mbar_init(&bars->p_full[x], 128);
+            mbar_init(&bars->o_full[x], 1);
+            mbar_init(&bars->o_empty[x], 128);
+        }
         mbar_init(&bars->final_mma, 1);
         bars->abort_flag = 0;
         fence_mbarrier_init();
@@ -203,29 +303,43 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            uint32_t g = 0;
-            for (int64_t item = blockIdx.x; item < items && !*abort_flag; item += gridDim.x) {
-                const TileInfo ti = decode_tile(a, item);
-                if (ti.kind < 0) continue;
-                const int64_t nst = tile_steps(ti);
-                const int64_t row0 = (int64_t)ti.b * a.N + ti.klo;
-                bool ok = true;
-                for (int64_t i = 0; i < nst; ++i, ++g) {
-                    const uint32_t s = g % TC_STAGES;
-                    if (!tc_wait(&bars->kv_empty[s], ((g / TC_STAGES) & 1) ^ 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* st = sKV + s * TC_STAGE_BYTES;
-                    mbar_arrive_expect_tx(&bars->kv_full[s], TC_STAGE_BYTES);
-                    const int r = (int)(row0 + i * MOBA_KCHUNK);
-                    tma_load_3d(smem_u32(st), &maps.k, &bars->kv_full[s], 0, ti.hk, r);
-                    tma_load_3d(smem_u32(st + 16384), &maps.k, &bars->kv_full[s], 64, ti.hk, r);
-                    tma_load_3d(smem_u32(st + 32768), &maps.v, &bars->kv_full[s], 0, ti.hk, r);
-                    tma_load_3d(smem_u32(st + 49152), &maps.v, &bars->kv_full[s], 64, ti.hk, r);
-                    bars->kv_issued[s] += 1;
+            uint32_t gk = 0, gv = 0;  // K and V steps issued so far
+            bool ok = true;
+            auto load = [&](bool is_v, int hk, int row) -> bool {
+                const uint32_t g = is_v ? gv : gk;
+                const uint32_t nslots = is_v ? TC_VSLOTS : TC_KSLOTS;
+                const uint32_t s = g % nslots;
+                uint64_t* full = is_v ? &bars->v_full[s] : &bars->k_full[s];
+                uint64_t* empty = is_v ? &bars->v_empty[s] : &bars->k_empty[s];
+                // completion #(g/n - 1) of the slot's empty barrier; #(g/n - 2) was waited n loads ago
+                ATRACE(is_v ? 2 : 0, g);  // producer: waiting for a slot
+                if (!tc_wait(empty, ((g / nslots) & 1) ^ 1, abort_flag, true)) return false;
+                ATRACE(is_v ? 3 : 1, g);  // producer: slot free, load issued
+                uint8_t* dst = (is_v ? sV : sK) + s * TC_STEP_BYTES;
+                const void* map = is_v ? (const void*)&maps.v : (const void*)&maps.k;
+                mbar_arrive_expect_tx(full, TC_STEP_BYTES);
+                tma_load_3d(smem_u32(dst), map, full, 0, hk, row);
+                tma_load_3d(smem_u32(dst + 16384), map, full, 64, hk, row);
+                if (is_v) {
+                    bars->v_issued[s] += 1;
+                    ++gv;
+                } else {
+                    bars->k_issued[s] += 1;
+                    ++gk;
                 }
-                if (!ok) break;
+                return true;
+            };
+            for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x) {
+                const PairInfo pi = decode_pair(a, item);
+                if (pi.ns == 0) continue;
+                const TileInfo& t0 = pi.t[0].kind >= 0 ? pi.t[0] : pi.t[1];
+                const int64_t row0 = (int64_t)t0.b * a.N + t0.klo;
+                // K one step ahead of V: K0, K1, V0, K2, V1, ...
+                if (!(ok = load(false, t0.hk, (int)row0))) break;
+                for (int64_t i = 0; i < pi.ns; ++i) {
+                    if (i + 1 < pi.ns && !(ok = load(false, t0.hk, (int)(row0 + (i + 1) * MOBA_KCHUNK)))) break;
+                    if (!(ok = load(true, t0.hk, (int)(row0 + i * MOBA_KCHUNK)))) break;
+                }
             }
         }
         __syncwarp();
@@ -234,59 +348,83 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (lane == 0) {
             const uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
             const uint32_t idesc_pv = make_idesc_bf16(128, 128, 0, 1);
-            const uint32_t sq = smem_u32(sQ), skv = smem_u32(sKV);
-            const uint32_t tO = tmem + 256;
-            uint32_t g = 0, tile_i = 0;
+            uint32_t gk = 0, gv = 0;                 // K / V steps consumed
+            uint32_t sx[2] = {0, 0}, px[2] = {0, 0}, tx[2] = {0, 0};  // per tile: Q K^T, P V, tiles issued
             bool ok = true;
-            auto issue_qk = [&](uint32_t gg) {
-                const uint32_t s = gg % TC_STAGES;
-                const uint32_t sk = skv + s * TC_STAGE_BYTES;
-                const uint32_t tS = tmem + (gg & 1) * 128;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                    tc_mma_ss(tS, make_sdesc_sw128(sq + off, 16, 1024), make_sdesc_sw128(sk + off, 16, 1024),
-                              idesc_qk, k > 0);
-                }
-                tc_commit(&bars->s_full[gg & 1]);
-            };
             for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x) {
-                const TileInfo ti = decode_tile(a, item);
-                if (ti.kind < 0) continue;
-                const uint32_t nst = (uint32_t)tile_steps(ti);
-                if (!(ok = tc_wait(&bars->q_full, tile_i & 1, abort_flag))) break;
-                tc_fence_after();
-                for (uint32_t i = 0; i < nst; ++i) {
-                    const uint32_t gg = g + i;
-                    if (i == 0) {
-                        if (!(ok = tc_wait(&bars->kv_full[gg % TC_STAGES], (gg / TC_STAGES) & 1, abort_flag))) break;
-                        tc_fence_after();
-                        issue_qk(gg);
-                    }
-                    if (i + 1 < nst) {
-                        const uint32_t g1 = gg + 1;
-                        if (!(ok = tc_wait(&bars->kv_full[g1 % TC_STAGES], (g1 / TC_STAGES) & 1, abort_flag))) break;
-                        tc_fence_after();
-                        issue_qk(g1);
-                    }
-                    if (!(ok = tc_wait(&bars->p_full[gg & 1], (gg >> 1) & 1, abort_flag))) break;
-                    tc_fence_after();
-                    if (i == 0) {
-                        if (!(ok = tc_wait(&bars->o_empty, (tile_i & 1) ^ 1, abort_flag))) break;
-                        tc_fence_after();
-                    }
-                    const uint32_t sv = skv + (gg % TC_STAGES) * TC_STAGE_BYTES + 32768;
-                    const uint32_t tP = tmem + (gg & 1) * 128;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        tc_mma_ts(tO, tP + k * 8, make_sdesc_sw128(sv + k * 2048, 16384, 1024), idesc_pv,
-                                  (i > 0 || k > 0) ? 1u : 0u);
-                    tc_commit(&bars->kv_empty[gg % TC_STAGES]);
-                    tc_commit(&bars->pv_done);
-                    if (i + 1 == nst) tc_commit(&bars->o_full);
+                const PairInfo pi = decode_pair(a, item);
+                if (pi.ns == 0) continue;
+                int64_t nst[2];
+                for (int x = 0; x < 2; ++x) {
+                    nst[x] = tile_steps(pi.t[x]);
+                    if (nst[x] == 0) continue;
+                    // completion #tx of q_full[x]: #tx-1 was waited for the previous tile of x
+                    if (!(ok = tc_wait(&bars->q_full[x], tx[x] & 1, abort_flag))) break;
                 }
-                g += nst;
-                tile_i += 1;
+                if (!ok) break;
+                tc_fence_after();
+                for (int64_t i = 0; i <= pi.ns && ok; ++i) {
+                    const bool do_qk = i < pi.ns;
+                    const bool do_pv = i > 0;
+                    uint32_t ks = 0, vs = 0;
+                    ATRACE(14, gk);  // MMA: iteration start
+                    if (do_qk) {
+                        ks = gk % TC_KSLOTS;
+                        if (!(ok = tc_wait(&bars->k_full[ks], (gk / TC_KSLOTS) & 1, abort_flag))) break;
+                    }
+                    ATRACE(15, gk);  // MMA: K ready
+                    if (do_pv) {
+                        vs = gv % TC_VSLOTS;
+                        if (!(ok = tc_wait(&bars->v_full[vs], (gv / TC_VSLOTS) & 1, abort_flag))) break;
+                    }
+                    ATRACE(16, gk);  // MMA: V ready
+                    tc_fence_after();
+                    for (int x = 0; x < 2 && ok; ++x) {
+                        const uint32_t tS = tmem + x * 128, tO = tmem + 256 + x * 128;
+                        if (do_pv && i - 1 < nst[x]) {
+                            // completion #px of p_full[x]; #px-1 was waited before the previous P V of x
+                            ATRACE(10 + x, px[x]);
+                            if (!(ok = tc_wait(&bars->p_full[x], px[x] & 1, abort_flag))) break;
+                            ATRACE(12 + x, px[x]);
+                            if (i == 1) {
+                                // O_x is free once the previous tile's epilogue has read it
+                                if (!(ok = tc_wait(&bars->o_empty[x], (tx[x] & 1) ^ 1, abort_flag))) break;
+                            }
+                            tc_fence_after();
+                            const uint32_t sv = smem_u32(sV + vs * TC_STEP_BYTES);
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                tc_mma_ts(tO, tS + 64 + k * 8, make_sdesc_sw128(sv + k * 2048, 16384, 1024), idesc_pv,
+                                          (i > 1 || k > 0) ? 1u : 0u);
+                            ++px[x];
+                            if (i == nst[x]) {  // that was the tile's last step
+                                tc_commit(&bars->o_full[x]);
+                                ++tx[x];
+                            }
+                        }
+                        if (do_qk && i < nst[x]) {
+                            const uint32_t sq = smem_u32(sQ + x * TC_Q_BYTES);
+                            const uint32_t sk = smem_u32(sK + ks * TC_STEP_BYTES);
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+                                tc_mma_ss(tS, make_sdesc_sw128(sq + off, 16, 1024),
+                                          make_sdesc_sw128(sk + off, 16, 1024), idesc_qk, k > 0);
+                            }
+                            tc_commit(&bars->s_full[x]);
+                            ++sx[x];
+                        }
+                    }
+                    if (!ok) break;
+                    if (do_qk) {
+                        tc_commit(&bars->k_empty[ks]);  // both tiles' Q K^T of this step read K
+                        ++gk;
+                    }
+                    if (do_pv) {
+                        tc_commit(&bars->v_empty[vs]);  // both tiles' P V of the previous step read V
+                        ++gv;
+                    }
+                }
             }
             // all MMAs issued by this thread have completed before TMEM is released
             tc_commit(&bars->final_mma);
@@ -295,12 +433,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax warps
-        const int r = 32 * (warp & 3) + lane;  // tile row == TMEM lane
+        const int x = (warp - 2) >> 2;           // tile of the pair handled by this warp group
+        const int r = 32 * (warp & 3) + lane;    // tile row == TMEM lane
         const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-        const uint32_t tO = tmem + 256 + lane_off;
+        const uint32_t tS = tmem + x * 128 + lane_off;
+        const uint32_t tO = tmem + 256 + x * 128 + lane_off;
+        uint8_t* sQx = sQ + x * TC_Q_BYTES;
         uint32_t g = 0, tile_i = 0;
         for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
-            const TileInfo ti = decode_tile(a, item);
+            const PairInfo pi = decode_pair(a, item);
+            const TileInfo& ti = pi.t[x];
             if (ti.kind < 0) continue;
             const uint32_t nst = (uint32_t)tile_steps(ti);
             // row identity
@@ -320,48 +462,65 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 t = ti.t0 + r;
                 hq = ti.hq;
             }
-            // gather this row of Q into the swizzled tile (zero rows past the end)
+            if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(30 + 50 * x, tile_i);
+            // gather this row of Q into the swizzled tile (zero rows past the end). The buffer is
+            // free: the previous tile's epilogue waited for its last P V, after every Q K^T of it.
             {
                 const uint16_t* src = a.q + (valid ? (((int64_t)ti.b * a.N + t) * a.Hq + hq) * MOBA_D : 0);
-                const uint32_t dst = smem_u32(sQ) + r * 128;
+                const uint32_t dst = smem_u32(sQx) + r * 128;
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
                     cp_async_16_zfill(dst + (c >> 3) * 16384 + (((c & 7) ^ (r & 7)) << 4), src + c * 8, valid);
                 cp_async_wait_all();
                 fence_proxy_async_smem();
-                mbar_arrive(&bars->q_full);
+                mbar_arrive(&bars->q_full[x]);
             }
             const int64_t tmask = ti.kind == 0 ? INT64_MAX : t;  // causal limit of the row
             float m_used = -INFINITY, l = 0.f;
             bool ok = true;
             for (uint32_t i = 0; i < nst; ++i) {
                 const uint32_t gg = g + i;
-                const uint32_t tS = tmem + (gg & 1) * 128 + lane_off;
-                if (!(ok = tc_wait_warp(&bars->s_full[gg & 1], (gg >> 1) & 1, abort_flag))) break;
+                if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(20 + 50 * x, gg);
+                // completion #gg of s_full[x]; #gg-1 was waited at the previous step
+                if (!(ok = tc_wait_warp(&bars->s_full[x], gg & 1, abort_flag))) break;
+                if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(21 + 50 * x, gg);
                 tc_fence_after();
-                uint32_t sr[4][32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
-                tc_wait_ld();
                 const int64_t u0 = ti.klo + (int64_t)i * MOBA_KCHUNK;
                 int64_t lim = ti.khi - 1 - u0;                 // last allowed column by the key range
                 if (tmask - u0 < lim) lim = tmask - u0;        // and by causality
-                if (lim < MOBA_KCHUNK - 1) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (c * 32 + j > lim) sr[c][j] = __float_as_uint(-INFINITY);
+                const bool full = lim >= MOBA_KCHUNK - 1;
+                // Optimistic pass: P against the current maximum. S columns [0,64) are read and
+                // their P computed, then columns [64,128) are read into registers, and only then
+                // is the first P stored over columns [64,96) (already read). If the step's maximum
+                // moved the running one, P is recomputed from S[0,64) (still in TMEM) and from the
+                // upper half still held in registers.
+                const float nm0 = (m_used == -INFINITY) ? 0.f : -m_used;
+                uint32_t s1[2][32];
+                float mx, lsum;
+                {
+                    uint32_t pk0[32];
+                    {
+                        uint32_t s0[2][32];
+                        tmem_ld32(tS, s0[0]);
+                        tmem_ld32(tS + 32, s0[1]);
+                        tc_wait_ld();
+                        if (!full) mask_cols(s0, 0, lim);
+                        mx = fmaxf(row_max32(s0[0]), row_max32(s0[1]));
+                        lsum = softmax_half(s0, pk0, a.scale_log2, nm0, full);
+                    }
+                    tmem_ld32(tS + 64, s1[0]);
+                    tmem_ld32(tS + 96, s1[1]);
+                    tc_wait_ld();
+                    tmem_st32(tS + 64, pk0);
                 }
-                const float mx = row_max128(sr);
+                if (!full) mask_cols(s1, 64, lim);
+                mx = fmaxf(mx, fmaxf(row_max32(s1[0]), row_max32(s1[1])));
                 const float m_new = fmaxf(m_used, mx * a.scale_log2);
-                const bool need = m_new > m_used + TC_RESCALE_LOG2;
-                if (__any_sync(0xffffffffu, need)) {
+                if (__any_sync(0xffffffffu, m_new > m_used + TC_RESCALE_LOG2)) {
+                    // the maximum moved (always on a tile's first step): rescale O and l, recompute P
                     const float f = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new);
-                    if (i > 0) {
-                        if (!(ok = tc_wait_warp(&bars->pv_done, (gg - 1) & 1, abort_flag))) break;
-                        tc_fence_after();
-#pragma unroll
+                    if (i > 0) {  // O_x holds P V of every earlier step (S ready implies it)
+#pragma unroll 1
                         for (int c = 0; c < 4; ++c) {
                             uint32_t o[32];
                             tmem_ld32(tO + c * 32, o);
@@ -374,96 +533,74 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     }
                     l *= f;
                     m_used = m_new;
-                }
-                const float nm = -m_used;
-                uint32_t pk[2][32];
-                if (lim >= MOBA_KCHUNK - 1) {
-                    // unmasked step: exponentials split between the MUFU and the FMA pipe
-                    const uint64_t sc2 = f2pack(a.scale_log2, a.scale_log2), nm2 = f2pack(nm, nm);
-                    uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-#pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
-                            const uint64_t x2 =
-                                ffma2(f2pack(__uint_as_float(sr[c][j]), __uint_as_float(sr[c][j + 1])), sc2, nm2);
-                            uint64_t p2;
-                            if (((j >> 1) & 7) < EXP2_POLY_PAIRS) {
-                                p2 = exp2_poly2(x2);
-                            } else {
-                                float x0, x1;
-                                f2unpack(x2, x0, x1);
-                                p2 = f2pack(ex2_approx(x0), ex2_approx(x1));
-                            }
-                            acc2[(j >> 1) & 3] = fadd2(acc2[(j >> 1) & 3], p2);
-                            float p0, p1;
-                            f2unpack(p2, p0, p1);
-                            pk[c >> 1][(c & 1) * 16 + (j >> 1)] = pack_bf16x2(p0, p1);
-                        }
-                    const uint64_t s2 = fadd2(fadd2(acc2[0], acc2[1]), fadd2(acc2[2], acc2[3]));
-                    float l0, l1;
-                    f2unpack(s2, l0, l1);
-                    l += l0 + l1;
+                    {  // upper half first, from registers, so they die before the lower half is reloaded
+                        uint32_t pk1[32];
+                        lsum = softmax_half(s1, pk1, a.scale_log2, -m_used, false);
+                        tmem_st32(tS + 96, pk1);
+                    }
+                    {
+                        uint32_t pk0[32];
+                        uint32_t s0[2][32];
+                        tmem_ld32(tS, s0[0]);
+                        tmem_ld32(tS + 32, s0[1]);
+                        tc_wait_ld();
+                        if (!full) mask_cols(s0, 0, lim);
+                        lsum += softmax_half(s0, pk0, a.scale_log2, -m_used, false);
+                        tmem_st32(tS + 64, pk0);
+                    }
                 } else {
-                    // masked step: MUFU only, so masked keys contribute exactly zero
-                    float ls[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) ls[u] = 0.f;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-#pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
-                            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][j]), a.scale_log2, nm));
-                            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][j + 1]), a.scale_log2, nm));
-                            pk[c >> 1][(c & 1) * 16 + (j >> 1)] = pack_bf16x2(p0, p1);
-                            ls[(j >> 1) & 7] += p0 + p1;
-                        }
-                    l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+                    uint32_t pk1[32];
+                    lsum += softmax_half(s1, pk1, a.scale_log2, nm0, full);
+                    tmem_st32(tS + 96, pk1);
                 }
-                tmem_st32(tS, pk[0]);
-                tmem_st32(tS + 32, pk[1]);
+                l += lsum;
                 tc_wait_st();
                 tc_fence_before();
-                mbar_arrive(&bars->p_full[gg & 1]);
+                mbar_arrive(&bars->p_full[x]);
+                if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(22 + 50 * x, gg);
             }
             if (!ok) break;
-            // epilogue. Waiting on pv_done here would be unsafe: the step barrier may still be two
-            // phases behind (the last Q K^T was issued before the previous P V), so the tile has
-            // its own barrier.
-            if (!tc_wait_warp(&bars->o_full, tile_i & 1, abort_flag)) break;
+            // epilogue: completion #tile_i of o_full[x]; #tile_i-1 was waited at the previous tile
+            if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(31 + 50 * x, tile_i);
+            if (!tc_wait_warp(&bars->o_full[x], tile_i & 1, abort_flag)) break;
             tc_fence_after();
-            uint32_t ob[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tO + c * 32, ob[c]);
-            tc_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&bars->o_empty);
-            if (valid) {
-                const float inv = 1.f / l;
-                const float lse = (m_used + __log2f(l)) * 0.69314718055994530942f;
-                uint16_t* dst;
-                float* ldst;
-                if (ti.kind == 0) {
-                    const int64_t prow = ((int64_t)ti.b * a.Hq + hq) * a.N + t;
-                    dst = a.opart + (prow * a.kp + slot) * MOBA_D;
-                    ldst = a.lpart + prow * a.kp + slot;
-                } else {
-                    dst = a.out + (((int64_t)ti.b * a.N + t) * a.Hq + hq) * MOBA_D;
-                    ldst = a.lse + ((int64_t)ti.b * a.Hq + hq) * a.N + t;
-                }
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-#pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(ob[c][j + 0]) * inv, __uint_as_float(ob[c][j + 1]) * inv);
-                        w.y = pack_bf16x2(__uint_as_float(ob[c][j + 2]) * inv, __uint_as_float(ob[c][j + 3]) * inv);
-                        w.z = pack_bf16x2(__uint_as_float(ob[c][j + 4]) * inv, __uint_as_float(ob[c][j + 5]) * inv);
-                        w.w = pack_bf16x2(__uint_as_float(ob[c][j + 6]) * inv, __uint_as_float(ob[c][j + 7]) * inv);
-                        *reinterpret_cast<uint4*>(dst + c * 32 + j) = w;
-                    }
-                *ldst = lse;
+            uint16_t* dst = nullptr;
+            float* ldst = nullptr;
+            if (ti.kind == 0) {
+                const int64_t prow = ((int64_t)ti.b * a.Hq + hq) * a.N + t;
+                dst = a.opart + (prow * a.kp + slot) * MOBA_D;
+                ldst = a.lpart + prow * a.kp + slot;
+            } else {
+                dst = a.out + (((int64_t)ti.b * a.N + t) * a.Hq + hq) * MOBA_D;
+                ldst = a.lse + ((int64_t)ti.b * a.Hq + hq) * a.N + t;
             }
+            const float inv = 1.f / l;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {  // 64 output features at a time
+                uint32_t ob[2][32];
+                tmem_ld32(tO + hh * 64, ob[0]);
+                tmem_ld32(tO + hh * 64 + 32, ob[1]);
+                tc_wait_ld();
+                if (hh == 1) {  // O_x has been read: the next tile may overwrite it
+                    tc_fence_before();
+                    mbar_arrive(&bars->o_empty[x]);
+                }
+                if (valid) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+#pragma unroll
+                        for (int j = 0; j < 32; j += 8) {
+                            uint4 w;
+                            w.x = pack_bf16x2(__uint_as_float(ob[c][j + 0]) * inv, __uint_as_float(ob[c][j + 1]) * inv);
+                            w.y = pack_bf16x2(__uint_as_float(ob[c][j + 2]) * inv, __uint_as_float(ob[c][j + 3]) * inv);
+                            w.z = pack_bf16x2(__uint_as_float(ob[c][j + 4]) * inv, __uint_as_float(ob[c][j + 5]) * inv);
+                            w.w = pack_bf16x2(__uint_as_float(ob[c][j + 6]) * inv, __uint_as_float(ob[c][j + 7]) * inv);
+                            *reinterpret_cast<uint4*>(dst + hh * 64 + c * 32 + j) = w;
+                        }
+                }
+            }
+            if (valid) *ldst = (m_used + __log2f(l)) * 0.69314718055994530942f;
+            if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(33 + 50 * x, tile_i);
             g += nst;
             tile_i += 1;
         }
@@ -473,10 +610,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     __syncthreads();
     if (warp == 0 && lane == 0 && *abort_flag) {
         // let every load already issued land before the shared memory goes away
-        for (int s = 0; s < TC_STAGES; ++s) {
-            const uint32_t n = bars->kv_issued[s];
-            if (n > 0) mbar_wait(&bars->kv_full[s], (n - 1) & 1);
-        }
+        for (int s = 0; s < TC_KSLOTS; ++s)
+            if (bars->k_issued[s] > 0) mbar_wait(&bars->k_full[s], (bars->k_issued[s] - 1) & 1);
+        for (int s = 0; s < TC_VSLOTS; ++s)
+            if (bars->v_issued[s] > 0) mbar_wait(&bars->v_full[s], (bars->v_issued[s] - 1) & 1);
     }
     tc_fence_before();
     __syncthreads();
@@ -526,10 +663,22 @@ static int run_attention_tc(const AttnParams& a, cudaStream_t st) {
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return MOBA_ERR_CUDA;
-    if (cudaFuncSetAttribute(moba_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_BYTES) !=
-        cudaSuccess)
-        return MOBA_ERR_CUDA;
-    const int64_t grid = items < nsm ? items : nsm;
+    {
+        const cudaError_t err =
+            cudaFuncSetAttribute(moba_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_BYTES);
+        if (err != cudaSuccess) {
+            moba_note_cuda_error(err);
+            return MOBA_ERR_CUDA;
+        }
+    }
+    const int64_t grid = items < nsm ? items : nsm;  // one CTA per SM, striped over the pairs
     moba_attn_tc_kernel<<<(unsigned)grid, TC_THREADS, TC_SMEM_BYTES, st>>>(a, maps, items);
-    return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA;
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) {
+        cudaGetLastError();
+        (void)cudaPeekAtLastError();
+        moba_note_cuda_error(err);
+        return MOBA_ERR_CUDA;
+    }
+    return MOBA_OK;
 }

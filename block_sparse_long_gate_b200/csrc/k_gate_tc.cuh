@@ -429,7 +429,14 @@ static int launch_gate_tc(const GateParams& gp, const GateMaps& maps, int grid, 
                              GATE_TC_SMEM) != cudaSuccess)
         return MOBA_ERR_CUDA;
     moba_gate_tc_kernel<KPX><<<grid, GATE_TC_THREADS, GATE_TC_SMEM, st>>>(gp, maps);
-    return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA;
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) {
+        cudaGetLastError();
+        (void)cudaPeekAtLastError();
+        moba_note_cuda_error(err);
+        return MOBA_ERR_CUDA;
+    }
+    return MOBA_OK;
 }
 
 static int run_gate_tc(const GateParams& gp, const uint16_t* planes, cudaStream_t st) {

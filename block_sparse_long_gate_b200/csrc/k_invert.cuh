@@ -112,8 +112,8 @@ __global__ void __launch_bounds__(INV_THREADS) moba_scatter_kernel(const int32_t
 #define SCAN_PER_THREAD 8
 #define SCAN_TILE (SCAN_THREADS * SCAN_PER_THREAD)
 
-// Value i of the scan input: either counts[i] or, for the tile counts, the
-// number of 128-row tiles of list i computed from the list offsets.
+// Value i of the scan input: either counts[i] or, for the work items, the
+// number of 256-row tile pairs of list i computed from the list offsets.
 struct ScanSrc {
     const uint32_t* vals;    // direct values, or null
     const int64_t* segoff;   // list offsets (stride nch) when vals is null
@@ -121,7 +121,7 @@ struct ScanSrc {
     __device__ __forceinline__ int64_t get(int64_t i) const {
         if (vals) return vals[i];
         int64_t len = segoff[(i + 1) * nch] - segoff[i * nch];
-        return (len + MOBA_TILE - 1) / MOBA_TILE;
+        return (len + 2 * MOBA_TILE - 1) / (2 * MOBA_TILE);
     }
 };
 

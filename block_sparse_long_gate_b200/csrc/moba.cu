@@ -69,6 +69,9 @@ struct StageTimer {
 
 inline void count_launch(int n = 1) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
+// Text of the last CUDA error the library saw on this host thread.
+thread_local const char* g_last_cuda_error = "no error";
+
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -107,11 +110,11 @@ int make_plan(int B, int Hq, int Hkv, int64_t N, int d, int bs, int topk, Plan* 
         per_head += n_c * (c < P.kp ? c : P.kp);
     }
     P.E = per_head * B * Hq;
-    P.Pmax = P.E / MOBA_TILE + P.L;
+    P.Pmax = P.E / MOBA_PAIR_ROWS + P.L;  // past pairs: <= 256 entries of one list each
     P.mb = cdiv(bs, MOBA_TILE);
     int64_t nlast = N - (P.nblk - 1) * bs;
     P.ml = cdiv(nlast, MOBA_TILE);
-    P.per_bh = (P.nblk - 1) * P.mb + P.ml;
+    P.per_bh = (P.nblk - 1) * cdiv(P.mb, 2) + cdiv(P.ml, 2);  // own-block pairs per (b, hq)
     P.D = (int64_t)B * Hq * P.per_bh;
     P.nseg = P.L * P.nch;
     int64_t nscan = P.nseg > P.L ? P.nseg : P.L;
@@ -168,7 +171,21 @@ int check_ptrs(std::initializer_list<const void*> ps) {
     return MOBA_OK;
 }
 
-int launch_ok() { return cudaGetLastError() == cudaSuccess ? MOBA_OK : MOBA_ERR_CUDA; }
+}  // namespace
+
+void moba_note_cuda_error(cudaError_t e) { g_last_cuda_error = cudaGetErrorString(e); }
+
+namespace {
+
+int cuda_fail(cudaError_t e) {
+    g_last_cuda_error = cudaGetErrorString(e);
+    return MOBA_ERR_CUDA;
+}
+
+int launch_ok() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MOBA_OK : cuda_fail(e);
+}
 
 // ---------------------------------------------------------------- stages
 // Gate scratch inside a workspace: Kbar (fp64) and, for the tensor-core gate, the centre /
@@ -325,6 +342,10 @@ int run_attention(const Plan& P, const AttnParams& a, cudaStream_t st) {
         return launch_ok();
     }
     const int rc = run_attention_tc(a, st);
+    if (rc == MOBA_ERR_CUDA) {
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) cuda_fail(e);
+    }
     if (rc == MOBA_OK && items > 0) count_launch();
     return rc;
 }
@@ -527,6 +548,8 @@ int moba_stage_times(float* ms, int n, int* calls) {
 
 uint64_t moba_launch_count(void) { return g_launches.load(); }
 
+const char* moba_last_error_string(void) { return g_last_cuda_error; }
+
 int moba_set_attention_impl(int impl) {
     int old = g_attn_impl;
     g_attn_impl = impl;
@@ -607,6 +630,15 @@ extern "C" int moba_debug_gate_stats(unsigned long long* out4, int reset) {
         unsigned long long z[4] = {0, 0, 0, 0};
         if (cudaMemcpyToSymbol(g_gate_stats, z, sizeof(z)) != cudaSuccess) return MOBA_ERR_CUDA;
     }
+    return MOBA_OK;
+}
+#endif
+
+#ifdef MOBA_ATTN_TRACE
+extern "C" int moba_debug_attn_trace(unsigned long long* dev_buf) {
+    unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_attn_trace, &dev_buf, sizeof(dev_buf)) != cudaSuccess) return MOBA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_attn_trace_n, &zero, sizeof(zero)) != cudaSuccess) return MOBA_ERR_CUDA;
     return MOBA_OK;
 }
 #endif

@@ -160,6 +160,10 @@ int moba_stage_times(float* ms, int n, int* calls);
 int moba_gate_noalloc(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv, int64_t N, int d,
                       int block_size, int topk, moba_stream_t stream);
 
+/* Text of the last CUDA runtime error the library met on the calling host thread
+ * (for messages after MOBA_ERR_CUDA); "no error" if there was none. Static string. */
+const char* moba_last_error_string(void);
+
 /* Number of kernels the library has launched in this process (all devices). */
 uint64_t moba_launch_count(void);
 
