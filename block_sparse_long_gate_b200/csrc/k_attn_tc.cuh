@@ -160,7 +160,7 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
 #define EXP2_POLY_PAIRS 3  // of every 8 pairs of a step, evaluated by exp2_poly2
 
 // Masks the columns of a 64-key half (first column index c0) beyond `lim`.
-__device__ __forceinline__ void mask_cols(uint32_t (&sr)[2][32], int c0, int64_t lim) {
+__device__ __forceinline__ void mask_cols(uint32_t (&sr)[2][32], int c0, int lim) {
 #pragma unroll
     for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -168,50 +168,35 @@ __device__ __forceinline__ void mask_cols(uint32_t (&sr)[2][32], int c0, int64_t
             if (c0 + c * 32 + j > lim) sr[c][j] = __float_as_uint(-INFINITY);
 }
 
-// P = exp2(s * scale - m) for 64 keys into 32 bf16 pairs; returns their fp32 sum.
-// `mixed` splits the exponentials between the MUFU and the FMA pipe (only for
-// unmasked keys: the FMA form clamps, the MUFU form gives exact zeros for -inf).
+// P = exp2(s * scale - m) for 64 keys into 32 bf16 pairs; returns their fp32 sum. The
+// exponentials are split between the MUFU (ex2.approx) and the FMA pipe (exp2_poly2). A masked
+// key (s = -inf) gets weight 0 on the MUFU path and 2^-126 on the FMA path (the clamp): next to
+// the row maximum's weight >= 1 that is far below fp32 resolution in l and in O.
 __device__ __forceinline__ float softmax_half(const uint32_t (&sr)[2][32], uint32_t (&pk)[32], float scale,
-                                              float nm, bool mixed) {
-    float lsum;
-    if (mixed) {
-        const uint64_t sc2 = f2pack(scale, scale), nm2 = f2pack(nm, nm);
-        uint64_t acc2[2] = {0ull, 0ull};
+                                              float nm) {
+    const uint64_t sc2 = f2pack(scale, scale), nm2 = f2pack(nm, nm);
+    uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+    for (int c = 0; c < 2; ++c)
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                const uint64_t x2 = ffma2(f2pack(__uint_as_float(sr[c][j]), __uint_as_float(sr[c][j + 1])), sc2, nm2);
-                uint64_t p2;
-                if (((j >> 1) & 7) < EXP2_POLY_PAIRS) {
-                    p2 = exp2_poly2(x2);
-                } else {
-                    float x0, x1;
-                    f2unpack(x2, x0, x1);
-                    p2 = f2pack(ex2_approx(x0), ex2_approx(x1));
-                }
-                acc2[(j >> 1) & 1] = fadd2(acc2[(j >> 1) & 1], p2);
-                float p0, p1;
-                f2unpack(p2, p0, p1);
-                pk[c * 16 + (j >> 1)] = pack_bf16x2(p0, p1);
+        for (int j = 0; j < 32; j += 2) {
+            const uint64_t x2 = ffma2(f2pack(__uint_as_float(sr[c][j]), __uint_as_float(sr[c][j + 1])), sc2, nm2);
+            uint64_t p2;
+            if (((j >> 1) & 7) < EXP2_POLY_PAIRS) {
+                p2 = exp2_poly2(x2);
+            } else {
+                float x0, x1;
+                f2unpack(x2, x0, x1);
+                p2 = f2pack(ex2_approx(x0), ex2_approx(x1));
             }
-        float l0, l1;
-        f2unpack(fadd2(acc2[0], acc2[1]), l0, l1);
-        lsum = l0 + l1;
-    } else {
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][j]), scale, nm));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][j + 1]), scale, nm));
-                pk[c * 16 + (j >> 1)] = pack_bf16x2(p0, p1);
-                ls[(j >> 1) & 3] += p0 + p1;
-            }
-        lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
-    }
-    return lsum;
+            acc2[(j >> 1) & 1] = fadd2(acc2[(j >> 1) & 1], p2);
+            float p0, p1;
+            f2unpack(p2, p0, p1);
+            pk[c * 16 + (j >> 1)] = pack_bf16x2(p0, p1);
+        }
+    float l0, l1;
+    f2unpack(fadd2(acc2[0], acc2[1]), l0, l1);
+    return l0 + l1;
 }
 
 // Bounded wait that also gives up when another role raised the abort flag.
@@ -238,18 +223,6 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, vol
     return __all_sync(0xffffffffu, ok);
 }
 
-#ifdef MOBA_ATTN_TRACE
-// Debug timeline of CTA 0 (debug builds only): slot [code][step] = clock64().
-__device__ unsigned long long* g_attn_trace;
-__device__ unsigned int g_attn_trace_n;
-#define ATRACE(code, step)                                                         \
-    do {                                                                           \
-        if (blockIdx.x == 0 && g_attn_trace && (step) < 4096u)                     \
-            g_attn_trace[(unsigned)(code) * 4096u + (unsigned)(step)] = clock64(); \
-    } while (0)
-#else
-#define ATRACE(code, step)
-#endif
 
 __global__ void __launch_bounds__(TC_THREADS, 1)
     moba_attn_tc_kernel(const AttnParams a, const __grid_constant__ TcMaps maps, int64_t items) {
@@ -312,9 +285,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 uint64_t* full = is_v ? &bars->v_full[s] : &bars->k_full[s];
                 uint64_t* empty = is_v ? &bars->v_empty[s] : &bars->k_empty[s];
                 // completion #(g/n - 1) of the slot's empty barrier; #(g/n - 2) was waited n loads ago
-                ATRACE(is_v ? 2 : 0, g);  // producer: waiting for a slot
                 if (!tc_wait(empty, ((g / nslots) & 1) ^ 1, abort_flag, true)) return false;
-                ATRACE(is_v ? 3 : 1, g);  // producer: slot free, load issued
                 uint8_t* dst = (is_v ? sV : sK) + s * TC_STEP_BYTES;
                 const void* map = is_v ? (const void*)&maps.v : (const void*)&maps.k;
                 mbar_arrive_expect_tx(full, TC_STEP_BYTES);
@@ -332,90 +303,85 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x) {
                 const PairInfo pi = decode_pair(a, item);
                 if (pi.ns == 0) continue;
-                const TileInfo& t0 = pi.t[0].kind >= 0 ? pi.t[0] : pi.t[1];
-                const int64_t row0 = (int64_t)t0.b * a.N + t0.klo;
+                const bool first = pi.t[0].kind >= 0;
+                const int hk = first ? pi.t[0].hk : pi.t[1].hk;
+                const int64_t row0 = (int64_t)(first ? pi.t[0].b : pi.t[1].b) * a.N + (first ? pi.t[0].klo : pi.t[1].klo);
                 // K one step ahead of V: K0, K1, V0, K2, V1, ...
-                if (!(ok = load(false, t0.hk, (int)row0))) break;
+                if (!(ok = load(false, hk, (int)row0))) break;
                 for (int64_t i = 0; i < pi.ns; ++i) {
-                    if (i + 1 < pi.ns && !(ok = load(false, t0.hk, (int)(row0 + (i + 1) * MOBA_KCHUNK)))) break;
-                    if (!(ok = load(true, t0.hk, (int)(row0 + i * MOBA_KCHUNK)))) break;
+                    if (i + 1 < pi.ns && !(ok = load(false, hk, (int)(row0 + (i + 1) * MOBA_KCHUNK)))) break;
+                    if (!(ok = load(true, hk, (int)(row0 + i * MOBA_KCHUNK)))) break;
                 }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Everything here lives in registers (no arrays indexed by the tile at run time):
+        // a local-memory access on this thread's critical path costs as much as a wait.
         if (lane == 0) {
             const uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
             const uint32_t idesc_pv = make_idesc_bf16(128, 128, 0, 1);
-            uint32_t gk = 0, gv = 0;                 // K / V steps consumed
-            uint32_t sx[2] = {0, 0}, px[2] = {0, 0}, tx[2] = {0, 0};  // per tile: Q K^T, P V, tiles issued
+            // descriptors of the first Q, K and V buffers; the others follow at fixed offsets
+            // (the start-address field is addr >> 4, and every buffer ends below 256 KB)
+            const uint64_t dq0 = make_sdesc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t dk0 = make_sdesc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t dv0 = make_sdesc_sw128(smem_u32(sV), 16384, 1024);
+            uint32_t gk = 0, gv = 0;                   // K / V steps consumed
+            uint32_t px0 = 0, px1 = 0, tx0 = 0, tx1 = 0;  // per tile: P V steps issued, tiles finished
             bool ok = true;
             for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x) {
                 const PairInfo pi = decode_pair(a, item);
                 if (pi.ns == 0) continue;
-                int64_t nst[2];
-                for (int x = 0; x < 2; ++x) {
-                    nst[x] = tile_steps(pi.t[x]);
-                    if (nst[x] == 0) continue;
-                    // completion #tx of q_full[x]: #tx-1 was waited for the previous tile of x
-                    if (!(ok = tc_wait(&bars->q_full[x], tx[x] & 1, abort_flag))) break;
-                }
-                if (!ok) break;
+                const int64_t n0 = tile_steps(pi.t[0]), n1 = tile_steps(pi.t[1]);
+                // completion #tx of q_full[x]: #tx-1 was waited for the previous tile of x
+                if (n0 > 0 && !(ok = tc_wait(&bars->q_full[0], tx0 & 1, abort_flag))) break;
+                if (n1 > 0 && !(ok = tc_wait(&bars->q_full[1], tx1 & 1, abort_flag))) break;
                 tc_fence_after();
                 for (int64_t i = 0; i <= pi.ns && ok; ++i) {
                     const bool do_qk = i < pi.ns;
                     const bool do_pv = i > 0;
-                    uint32_t ks = 0, vs = 0;
-                    ATRACE(14, gk);  // MMA: iteration start
-                    if (do_qk) {
-                        ks = gk % TC_KSLOTS;
-                        if (!(ok = tc_wait(&bars->k_full[ks], (gk / TC_KSLOTS) & 1, abort_flag))) break;
-                    }
-                    ATRACE(15, gk);  // MMA: K ready
-                    if (do_pv) {
-                        vs = gv % TC_VSLOTS;
-                        if (!(ok = tc_wait(&bars->v_full[vs], (gv / TC_VSLOTS) & 1, abort_flag))) break;
-                    }
-                    ATRACE(16, gk);  // MMA: V ready
-                    tc_fence_after();
-                    for (int x = 0; x < 2 && ok; ++x) {
+                    const uint32_t ks = gk % TC_KSLOTS, vs = gv % TC_VSLOTS;
+                    const uint64_t kd = dk0 + (uint64_t)(ks * (TC_STEP_BYTES >> 4));
+                    const uint64_t vd = dv0 + (uint64_t)(vs * (TC_STEP_BYTES >> 4));
+                    if (do_pv && !(ok = tc_wait(&bars->v_full[vs], (gv / TC_VSLOTS) & 1, abort_flag))) break;
+                    bool k_ready = false;
+                    // One tile's work of this iteration: P V for step i - 1, then Q K^T for step i.
+                    auto tile = [&](const int x, const int64_t nx, uint32_t& pxx, uint32_t& txx) -> bool {
                         const uint32_t tS = tmem + x * 128, tO = tmem + 256 + x * 128;
-                        if (do_pv && i - 1 < nst[x]) {
-                            // completion #px of p_full[x]; #px-1 was waited before the previous P V of x
-                            ATRACE(10 + x, px[x]);
-                            if (!(ok = tc_wait(&bars->p_full[x], px[x] & 1, abort_flag))) break;
-                            ATRACE(12 + x, px[x]);
-                            if (i == 1) {
-                                // O_x is free once the previous tile's epilogue has read it
-                                if (!(ok = tc_wait(&bars->o_empty[x], (tx[x] & 1) ^ 1, abort_flag))) break;
-                            }
+                        if (do_pv && i - 1 < nx) {
+                            // completion #pxx of p_full[x]; #pxx-1 was waited before the previous P V of x
+                            if (!tc_wait(&bars->p_full[x], pxx & 1, abort_flag)) return false;
+                            // O_x is free once the previous tile's epilogue has read it
+                            if (i == 1 && !tc_wait(&bars->o_empty[x], (txx & 1) ^ 1, abort_flag)) return false;
                             tc_fence_after();
-                            const uint32_t sv = smem_u32(sV + vs * TC_STEP_BYTES);
+                            tc_mma_ts(tO, tS + 64, vd, idesc_pv, i > 1 ? 1u : 0u);
 #pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                tc_mma_ts(tO, tS + 64 + k * 8, make_sdesc_sw128(sv + k * 2048, 16384, 1024), idesc_pv,
-                                          (i > 1 || k > 0) ? 1u : 0u);
-                            ++px[x];
-                            if (i == nst[x]) {  // that was the tile's last step
+                            for (int k = 1; k < 8; ++k) tc_mma_ts(tO, tS + 64 + k * 8, vd + k * 128, idesc_pv, 1u);
+                            ++pxx;
+                            if (i == nx) {  // that was the tile's last step
                                 tc_commit(&bars->o_full[x]);
-                                ++tx[x];
+                                ++txx;
                             }
                         }
-                        if (do_qk && i < nst[x]) {
-                            const uint32_t sq = smem_u32(sQ + x * TC_Q_BYTES);
-                            const uint32_t sk = smem_u32(sK + ks * TC_STEP_BYTES);
+                        if (do_qk && i < nx) {
+                            if (!k_ready) {
+                                if (!tc_wait(&bars->k_full[ks], (gk / TC_KSLOTS) & 1, abort_flag)) return false;
+                                tc_fence_after();
+                                k_ready = true;
+                            }
+                            const uint64_t qd = dq0 + (uint64_t)(x * (TC_Q_BYTES >> 4));
 #pragma unroll
                             for (int k = 0; k < 8; ++k) {
-                                const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                                tc_mma_ss(tS, make_sdesc_sw128(sq + off, 16, 1024),
-                                          make_sdesc_sw128(sk + off, 16, 1024), idesc_qk, k > 0);
+                                const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+                                tc_mma_ss(tS, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
                             }
                             tc_commit(&bars->s_full[x]);
-                            ++sx[x];
                         }
-                    }
-                    if (!ok) break;
+                        return true;
+                    };
+                    if (!(ok = tile(0, n0, px0, tx0))) break;
+                    if (!(ok = tile(1, n1, px1, tx1))) break;
                     if (do_qk) {
                         tc_commit(&bars->k_empty[ks]);  // both tiles' Q K^T of this step read K
                         ++gk;
@@ -442,7 +408,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         uint32_t g = 0, tile_i = 0;
         for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
             const PairInfo pi = decode_pair(a, item);
-            const TileInfo& ti = pi.t[x];
+            const TileInfo ti = x ? pi.t[1] : pi.t[0];  // by value: stays in registers
             if (ti.kind < 0) continue;
             const uint32_t nst = (uint32_t)tile_steps(ti);
             // row identity
@@ -462,7 +428,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 t = ti.t0 + r;
                 hq = ti.hq;
             }
-            if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(30 + 50 * x, tile_i);
             // gather this row of Q into the swizzled tile (zero rows past the end). The buffer is
             // free: the previous tile's epilogue waited for its last P V, after every Q K^T of it.
             {
@@ -475,51 +440,83 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 fence_proxy_async_smem();
                 mbar_arrive(&bars->q_full[x]);
             }
-            const int64_t tmask = ti.kind == 0 ? INT64_MAX : t;  // causal limit of the row
+            // last key column this row may read, relative to the tile's first key: the key range
+            // and, on the own block, causality (u <= t)
+            int lim0;
+            {
+                int64_t last = ti.khi - 1;
+                if (ti.kind != 0 && t < last) last = t;
+                lim0 = (int)(last - ti.klo);
+            }
+            // output row: the slot's partial for a past tile, out / lse for an own-block tile
+            uint16_t* dst;
+            float* ldst;
+            if (ti.kind == 0) {
+                const int64_t prow = ((int64_t)ti.b * a.Hq + hq) * a.N + t;
+                dst = a.opart + (prow * a.kp + slot) * MOBA_D;
+                ldst = a.lpart + prow * a.kp + slot;
+            } else {
+                dst = a.out + (((int64_t)ti.b * a.N + t) * a.Hq + hq) * MOBA_D;
+                ldst = a.lse + ((int64_t)ti.b * a.Hq + hq) * a.N + t;
+            }
             float m_used = -INFINITY, l = 0.f;
             bool ok = true;
             for (uint32_t i = 0; i < nst; ++i) {
                 const uint32_t gg = g + i;
-                if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(20 + 50 * x, gg);
                 // completion #gg of s_full[x]; #gg-1 was waited at the previous step
                 if (!(ok = tc_wait_warp(&bars->s_full[x], gg & 1, abort_flag))) break;
-                if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(21 + 50 * x, gg);
                 tc_fence_after();
-                const int64_t u0 = ti.klo + (int64_t)i * MOBA_KCHUNK;
-                int64_t lim = ti.khi - 1 - u0;                 // last allowed column by the key range
-                if (tmask - u0 < lim) lim = tmask - u0;        // and by causality
+                const int lim = lim0 - (int)i * MOBA_KCHUNK;  // last allowed column of this step
                 const bool full = lim >= MOBA_KCHUNK - 1;
-                // Optimistic pass: P against the current maximum. S columns [0,64) are read and
-                // their P computed, then columns [64,128) are read into registers, and only then
-                // is the first P stored over columns [64,96) (already read). If the step's maximum
-                // moved the running one, P is recomputed from S[0,64) (still in TMEM) and from the
-                // upper half still held in registers.
-                const float nm0 = (m_used == -INFINITY) ? 0.f : -m_used;
-                uint32_t s1[2][32];
-                float mx, lsum;
-                {
-                    uint32_t pk0[32];
-                    {
-                        uint32_t s0[2][32];
-                        tmem_ld32(tS, s0[0]);
-                        tmem_ld32(tS + 32, s0[1]);
-                        tc_wait_ld();
-                        if (!full) mask_cols(s0, 0, lim);
-                        mx = fmaxf(row_max32(s0[0]), row_max32(s0[1]));
-                        lsum = softmax_half(s0, pk0, a.scale_log2, nm0, full);
-                    }
-                    tmem_ld32(tS + 64, s1[0]);
-                    tmem_ld32(tS + 96, s1[1]);
+                if (i == 0) {
+                    // The running maximum starts at the first step's row maximum (finite: column 0
+                    // of a tile's first step is allowed for every row), so that step never rescales.
+                    uint32_t sm[2][32];
+                    tmem_ld32(tS, sm[0]);
+                    tmem_ld32(tS + 32, sm[1]);
                     tc_wait_ld();
-                    tmem_st32(tS + 64, pk0);
+                    if (!full) mask_cols(sm, 0, lim);
+                    float mx = fmaxf(row_max32(sm[0]), row_max32(sm[1]));
+                    tmem_ld32(tS + 64, sm[0]);
+                    tmem_ld32(tS + 96, sm[1]);
+                    tc_wait_ld();
+                    if (!full) mask_cols(sm, 64, lim);
+                    mx = fmaxf(mx, fmaxf(row_max32(sm[0]), row_max32(sm[1])));
+                    m_used = mx * a.scale_log2;
                 }
-                if (!full) mask_cols(s1, 64, lim);
-                mx = fmaxf(mx, fmaxf(row_max32(s1[0]), row_max32(s1[1])));
-                const float m_new = fmaxf(m_used, mx * a.scale_log2);
-                if (__any_sync(0xffffffffu, m_new > m_used + TC_RESCALE_LOG2)) {
-                    // the maximum moved (always on a tile's first step): rescale O and l, recompute P
-                    const float f = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - m_new);
-                    if (i > 0) {  // O_x holds P V of every earlier step (S ready implies it)
+                // P against the running maximum. S columns [0,64) are read and their P computed,
+                // then columns [64,128) are read into registers, and only then is the first P
+                // stored over columns [64,96) (already read). If the step's maximum moved the
+                // running one by more than the threshold, the overwritten S columns are put back
+                // from registers, O and l are rescaled and the step is done again (rare: the
+                // first step already fixed the scale).
+                for (;;) {
+                    const float nm = -m_used;
+                    uint32_t s1[2][32];
+                    float mx, lsum;
+                    {
+                        uint32_t pk0[32];
+                        {
+                            uint32_t s0[2][32];
+                            tmem_ld32(tS, s0[0]);
+                            tmem_ld32(tS + 32, s0[1]);
+                            tc_wait_ld();
+                            if (!full) mask_cols(s0, 0, lim);
+                            mx = fmaxf(row_max32(s0[0]), row_max32(s0[1]));
+                            lsum = softmax_half(s0, pk0, a.scale_log2, nm);
+                        }
+                        tmem_ld32(tS + 64, s1[0]);
+                        tmem_ld32(tS + 96, s1[1]);
+                        tc_wait_ld();
+                        tmem_st32(tS + 64, pk0);
+                    }
+                    if (!full) mask_cols(s1, 64, lim);
+                    mx = fmaxf(mx, fmaxf(row_max32(s1[0]), row_max32(s1[1])));
+                    const float m_new = fmaxf(m_used, mx * a.scale_log2);
+                    if (__any_sync(0xffffffffu, m_new > m_used + TC_RESCALE_LOG2)) {
+                        tmem_st32(tS + 64, s1[0]);  // S columns [64,96) again (masked ones stay masked)
+                        const float f = ex2_approx(m_used - m_new);
+                        // O_x holds P V of every earlier step (S ready implies it); i > 0 here
 #pragma unroll 1
                         for (int c = 0; c < 4; ++c) {
                             uint32_t o[32];
@@ -529,53 +526,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                             for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
                             tmem_st32(tO + c * 32, o);
                         }
-                        tc_wait_st();
+                        l *= f;
+                        m_used = m_new;
+                        tc_wait_st();  // the restored S columns land before they are read again
+                        continue;
                     }
-                    l *= f;
-                    m_used = m_new;
-                    {  // upper half first, from registers, so they die before the lower half is reloaded
-                        uint32_t pk1[32];
-                        lsum = softmax_half(s1, pk1, a.scale_log2, -m_used, false);
-                        tmem_st32(tS + 96, pk1);
-                    }
-                    {
-                        uint32_t pk0[32];
-                        uint32_t s0[2][32];
-                        tmem_ld32(tS, s0[0]);
-                        tmem_ld32(tS + 32, s0[1]);
-                        tc_wait_ld();
-                        if (!full) mask_cols(s0, 0, lim);
-                        lsum += softmax_half(s0, pk0, a.scale_log2, -m_used, false);
-                        tmem_st32(tS + 64, pk0);
-                    }
-                } else {
                     uint32_t pk1[32];
-                    lsum += softmax_half(s1, pk1, a.scale_log2, nm0, full);
+                    lsum += softmax_half(s1, pk1, a.scale_log2, nm);
                     tmem_st32(tS + 96, pk1);
+                    l += lsum;
+                    break;
                 }
-                l += lsum;
                 tc_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bars->p_full[x]);
-                if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(22 + 50 * x, gg);
             }
             if (!ok) break;
             // epilogue: completion #tile_i of o_full[x]; #tile_i-1 was waited at the previous tile
-            if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(31 + 50 * x, tile_i);
             if (!tc_wait_warp(&bars->o_full[x], tile_i & 1, abort_flag)) break;
             tc_fence_after();
-            uint16_t* dst = nullptr;
-            float* ldst = nullptr;
-            if (ti.kind == 0) {
-                const int64_t prow = ((int64_t)ti.b * a.Hq + hq) * a.N + t;
-                dst = a.opart + (prow * a.kp + slot) * MOBA_D;
-                ldst = a.lpart + prow * a.kp + slot;
-            } else {
-                dst = a.out + (((int64_t)ti.b * a.N + t) * a.Hq + hq) * MOBA_D;
-                ldst = a.lse + ((int64_t)ti.b * a.Hq + hq) * a.N + t;
-            }
             const float inv = 1.f / l;
-#pragma unroll
+#pragma unroll 1
             for (int hh = 0; hh < 2; ++hh) {  // 64 output features at a time
                 uint32_t ob[2][32];
                 tmem_ld32(tO + hh * 64, ob[0]);
@@ -600,7 +571,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 }
             }
             if (valid) *ldst = (m_used + __log2f(l)) * 0.69314718055994530942f;
-            if (lane == 0 && (warp == 2 || warp == 6)) ATRACE(33 + 50 * x, tile_i);
             g += nst;
             tile_i += 1;
         }

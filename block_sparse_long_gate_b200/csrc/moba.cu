@@ -634,11 +634,3 @@ extern "C" int moba_debug_gate_stats(unsigned long long* out4, int reset) {
 }
 #endif
 
-#ifdef MOBA_ATTN_TRACE
-extern "C" int moba_debug_attn_trace(unsigned long long* dev_buf) {
-    unsigned zero = 0;
-    if (cudaMemcpyToSymbol(g_attn_trace, &dev_buf, sizeof(dev_buf)) != cudaSuccess) return MOBA_ERR_CUDA;
-    if (cudaMemcpyToSymbol(g_attn_trace_n, &zero, sizeof(zero)) != cudaSuccess) return MOBA_ERR_CUDA;
-    return MOBA_OK;
-}
-#endif
