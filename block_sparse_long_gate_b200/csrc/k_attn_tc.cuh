@@ -317,85 +317,86 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // Everything here lives in registers (no arrays indexed by the tile at run time):
-        // a local-memory access on this thread's critical path costs as much as a wait.
-        if (lane == 0) {
-            const uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
-            const uint32_t idesc_pv = make_idesc_bf16(128, 128, 0, 1);
-            // descriptors of the first Q, K and V buffers; the others follow at fixed offsets
-            // (the start-address field is addr >> 4, and every buffer ends below 256 KB)
-            const uint64_t dq0 = make_sdesc_sw128(smem_u32(sQ), 16, 1024);
-            const uint64_t dk0 = make_sdesc_sw128(smem_u32(sK), 16, 1024);
-            const uint64_t dv0 = make_sdesc_sw128(smem_u32(sV), 16384, 1024);
-            uint32_t gk = 0, gv = 0;                   // K / V steps consumed
-            uint32_t px0 = 0, px1 = 0, tx0 = 0, tx1 = 0;  // per tile: P V steps issued, tiles finished
-            bool ok = true;
-            for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x) {
-                const PairInfo pi = decode_pair(a, item);
-                if (pi.ns == 0) continue;
-                const int64_t n0 = tile_steps(pi.t[0]), n1 = tile_steps(pi.t[1]);
-                // completion #tx of q_full[x]: #tx-1 was waited for the previous tile of x
-                if (n0 > 0 && !(ok = tc_wait(&bars->q_full[0], tx0 & 1, abort_flag))) break;
-                if (n1 > 0 && !(ok = tc_wait(&bars->q_full[1], tx1 & 1, abort_flag))) break;
-                tc_fence_after();
-                for (int64_t i = 0; i <= pi.ns && ok; ++i) {
-                    const bool do_qk = i < pi.ns;
-                    const bool do_pv = i > 0;
-                    const uint32_t ks = gk % TC_KSLOTS, vs = gv % TC_VSLOTS;
-                    const uint64_t kd = dk0 + (uint64_t)(ks * (TC_STEP_BYTES >> 4));
-                    const uint64_t vd = dv0 + (uint64_t)(vs * (TC_STEP_BYTES >> 4));
-                    if (do_pv && !(ok = tc_wait(&bars->v_full[vs], (gv / TC_VSLOTS) & 1, abort_flag))) break;
-                    bool k_ready = false;
-                    // One tile's work of this iteration: P V for step i - 1, then Q K^T for step i.
-                    auto tile = [&](const int x, const int64_t nx, uint32_t& pxx, uint32_t& txx) -> bool {
-                        const uint32_t tS = tmem + x * 128, tO = tmem + 256 + x * 128;
-                        if (do_pv && i - 1 < nx) {
-                            // completion #pxx of p_full[x]; #pxx-1 was waited before the previous P V of x
-                            if (!tc_wait(&bars->p_full[x], pxx & 1, abort_flag)) return false;
-                            // O_x is free once the previous tile's epilogue has read it
-                            if (i == 1 && !tc_wait(&bars->o_empty[x], (txx & 1) ^ 1, abort_flag)) return false;
+        // The whole warp runs this loop, converged, so every descriptor and counter is
+        // warp-uniform; each MMA and commit is issued by the elected lane (always lane 0 of the
+        // full warp, so a commit covers every MMA before it). Nothing here is an array indexed
+        // at run time: a local-memory access on this critical path costs as much as a wait.
+        const uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
+        const uint32_t idesc_pv = make_idesc_bf16(128, 128, 0, 1);
+        // descriptors of the first Q, K and V buffers; the others follow at fixed offsets
+        // (the start-address field is addr >> 4, and every buffer ends below 256 KB)
+        const uint64_t dq0 = make_sdesc_sw128(smem_u32(sQ), 16, 1024);
+        const uint64_t dk0 = make_sdesc_sw128(smem_u32(sK), 16, 1024);
+        const uint64_t dv0 = make_sdesc_sw128(smem_u32(sV), 16384, 1024);
+        uint32_t gk = 0, gv = 0;                      // K / V steps consumed
+        uint32_t px0 = 0, px1 = 0, tx0 = 0, tx1 = 0;  // per tile: P V steps issued, tiles finished
+        bool ok = true;
+        for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x) {
+            const PairInfo pi = decode_pair(a, item);
+            if (pi.ns == 0) continue;
+            const int64_t n0 = tile_steps(pi.t[0]), n1 = tile_steps(pi.t[1]);
+            // completion #tx of q_full[x]: #tx-1 was waited for the previous tile of x
+            if (n0 > 0 && !(ok = tc_wait_warp(&bars->q_full[0], tx0 & 1, abort_flag))) break;
+            if (n1 > 0 && !(ok = tc_wait_warp(&bars->q_full[1], tx1 & 1, abort_flag))) break;
+            tc_fence_after();
+            for (int64_t i = 0; i <= pi.ns && ok; ++i) {
+                const bool do_qk = i < pi.ns;
+                const bool do_pv = i > 0;
+                const uint32_t ks = gk % TC_KSLOTS, vs = gv % TC_VSLOTS;
+                const uint64_t kd = dk0 + (uint64_t)(ks * (TC_STEP_BYTES >> 4));
+                const uint64_t vd = dv0 + (uint64_t)(vs * (TC_STEP_BYTES >> 4));
+                if (do_pv && !(ok = tc_wait_warp(&bars->v_full[vs], (gv / TC_VSLOTS) & 1, abort_flag))) break;
+                bool k_ready = false;
+                // One tile's work of this iteration: P V for step i - 1, then Q K^T for step i.
+                auto tile = [&](const int x, const int64_t nx, uint32_t& pxx, uint32_t& txx) -> bool {
+                    const uint32_t tS = tmem + x * 128, tO = tmem + 256 + x * 128;
+                    if (do_pv && i - 1 < nx) {
+                        // completion #pxx of p_full[x]; #pxx-1 was waited before the previous P V of x
+                        if (!tc_wait_warp(&bars->p_full[x], pxx & 1, abort_flag)) return false;
+                        // O_x is free once the previous tile's epilogue has read it
+                        if (i == 1 && !tc_wait_warp(&bars->o_empty[x], (txx & 1) ^ 1, abort_flag)) return false;
+                        tc_fence_after();
+                        tc_mma_ts_w(tO, tS + 64, vd, idesc_pv, i > 1 ? 1u : 0u);
+#pragma unroll
+                        for (int k = 1; k < 8; ++k) tc_mma_ts_w(tO, tS + 64 + k * 8, vd + k * 128, idesc_pv, 1u);
+                        ++pxx;
+                        if (i == nx) {  // that was the tile's last step
+                            tc_commit_w(&bars->o_full[x]);
+                            ++txx;
+                        }
+                    }
+                    if (do_qk && i < nx) {
+                        if (!k_ready) {
+                            if (!tc_wait_warp(&bars->k_full[ks], (gk / TC_KSLOTS) & 1, abort_flag)) return false;
                             tc_fence_after();
-                            tc_mma_ts(tO, tS + 64, vd, idesc_pv, i > 1 ? 1u : 0u);
-#pragma unroll
-                            for (int k = 1; k < 8; ++k) tc_mma_ts(tO, tS + 64 + k * 8, vd + k * 128, idesc_pv, 1u);
-                            ++pxx;
-                            if (i == nx) {  // that was the tile's last step
-                                tc_commit(&bars->o_full[x]);
-                                ++txx;
-                            }
+                            k_ready = true;
                         }
-                        if (do_qk && i < nx) {
-                            if (!k_ready) {
-                                if (!tc_wait(&bars->k_full[ks], (gk / TC_KSLOTS) & 1, abort_flag)) return false;
-                                tc_fence_after();
-                                k_ready = true;
-                            }
-                            const uint64_t qd = dq0 + (uint64_t)(x * (TC_Q_BYTES >> 4));
+                        const uint64_t qd = dq0 + (uint64_t)(x * (TC_Q_BYTES >> 4));
 #pragma unroll
-                            for (int k = 0; k < 8; ++k) {
-                                const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
-                                tc_mma_ss(tS, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
-                            }
-                            tc_commit(&bars->s_full[x]);
+                        for (int k = 0; k < 8; ++k) {
+                            const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+                            tc_mma_ss_w(tS, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
                         }
-                        return true;
-                    };
-                    if (!(ok = tile(0, n0, px0, tx0))) break;
-                    if (!(ok = tile(1, n1, px1, tx1))) break;
-                    if (do_qk) {
-                        tc_commit(&bars->k_empty[ks]);  // both tiles' Q K^T of this step read K
-                        ++gk;
+                        tc_commit_w(&bars->s_full[x]);
                     }
-                    if (do_pv) {
-                        tc_commit(&bars->v_empty[vs]);  // both tiles' P V of the previous step read V
-                        ++gv;
-                    }
+                    return true;
+                };
+                if (!(ok = tile(0, n0, px0, tx0))) break;
+                if (!(ok = tile(1, n1, px1, tx1))) break;
+                if (do_qk) {
+                    tc_commit_w(&bars->k_empty[ks]);  // both tiles' Q K^T of this step read K
+                    ++gk;
+                }
+                if (do_pv) {
+                    tc_commit_w(&bars->v_empty[vs]);  // both tiles' P V of the previous step read V
+                    ++gv;
                 }
             }
-            // all MMAs issued by this thread have completed before TMEM is released
-            tc_commit(&bars->final_mma);
-            mbar_wait(&bars->final_mma, 0);
         }
+        // all MMAs issued by the elected lane have completed before TMEM is released
+        __syncwarp();
+        tc_commit_w(&bars->final_mma);
+        mbar_wait(&bars->final_mma, 0);
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax warps
