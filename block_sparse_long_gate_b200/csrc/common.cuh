@@ -27,6 +27,14 @@ void moba_note_cuda_error(cudaError_t e);
 // records MOBA_ERR_DEVICE_TIMEOUT and the kernel leaves the wait. With the
 // nanosleep back-off below this is several seconds of waiting.
 #define MOBA_SPIN_LIMIT (1u << 26)
+// Wall-clock limit (ns, %globaltimer) of the waits that spin without back-off.
+#define MOBA_WAIT_NS 2000000000ull
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
     return __uint_as_float(((uint32_t)h) << 16);
@@ -192,6 +200,15 @@ __device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
         "elect.sync _|e, 0xffffffff;\n\t"
         "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
             smem_u32(bar))
+        : "memory");
+}
+
+// Plain arrive (count 1) by the elected lane of a converged warp.
+__device__ __forceinline__ void mbar_arrive_w(uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b64 st;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
         : "memory");
 }
 

@@ -42,7 +42,7 @@
 
 #include "k_attn_common.cuh"
 
-#define TC_THREADS 320
+#define TC_THREADS 352
 #define TC_KSLOTS 3
 #define TC_VSLOTS 2
 #define TC_STEP_BYTES 32768  // one K or V step: 128 keys x 128 d x bf16
@@ -63,7 +63,7 @@ struct TcBars {
     uint64_t p_full[2];   // per tile: P_X of a step is in TMEM
     uint64_t o_full[2];   // per tile: the tile's last P V is in O_X
     uint64_t o_empty[2];  // per tile: the epilogue has read O_X
-    uint64_t final_mma;
+    uint64_t final_mma[2];  // per issuer: all of its MMAs have completed
     uint32_t tmem_base;
     int abort_flag;
     uint32_t k_issued[TC_KSLOTS], v_issued[TC_VSLOTS];  // loads issued per slot (teardown bookkeeping)
@@ -202,15 +202,22 @@ __device__ __forceinline__ float softmax_half(const uint32_t (&sr)[2][32], uint3
 // Bounded wait that also gives up when another role raised the abort flag.
 // `backoff` adds a short sleep between polls (for roles off the critical path,
 // so their spinning does not take issue slots from the softmax warps).
+// The limit is wall-clock time (MOBA_WAIT_NS), read every 256 polls.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                         bool backoff = false) {
     uint32_t n = 0;
+    uint64_t t0 = 0;
     while (!mbar_try_wait(bar, parity)) {
         if (*abort_flag) return false;
-        if (++n >= MOBA_SPIN_LIMIT) {
-            moba_set_error(MOBA_ERR_DEVICE_TIMEOUT);
-            *abort_flag = 1;
-            return false;
+        if ((++n & 255) == 0) {
+            const uint64_t now = global_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > MOBA_WAIT_NS) {
+                moba_set_error(MOBA_ERR_DEVICE_TIMEOUT);
+                *abort_flag = 1;
+                return false;
+            }
         }
         if (backoff) __nanosleep(128);
     }
@@ -241,12 +248,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < TC_KSLOTS; ++s) {
             mbar_init(&bars->k_full[s], 1);
-            mbar_init(&bars->k_empty[s], 1);
+            mbar_init(&bars->k_empty[s], 2);  // one arrival per MMA issuer
             bars->k_issued[s] = 0;
         }
         for (int s = 0; s < TC_VSLOTS; ++s) {
             mbar_init(&bars->v_full[s], 1);
-            mbar_init(&bars->v_empty[s], 1);
+            mbar_init(&bars->v_empty[s], 2);
             bars->v_issued[s] = 0;
         }
         for (int x = 0; x < 2; ++x) {
@@ -256,7 +263,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             mbar_init(&bars->o_full[x], 1);
             mbar_init(&bars->o_empty[x], 128);
         }
-        mbar_init(&bars->final_mma, 1);
+        mbar_init(&bars->final_mma[0], 1);
+        mbar_init(&bars->final_mma[1], 1);
         bars->abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -315,88 +323,87 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        // The whole warp runs this loop, converged, so every descriptor and counter is
-        // warp-uniform; each MMA and commit is issued by the elected lane (always lane 0 of the
-        // full warp, so a commit covers every MMA before it). Nothing here is an array indexed
-        // at run time: a local-memory access on this critical path costs as much as a wait.
+    } else if (warp == 1 || warp == TC_THREADS / 32 - 1) {
+        // ------------------------------------------------------------ MMA issuers
+        // One warp per tile (warp 1: tile A, the last warp: tile B), so each tile's P V and
+        // Q K^T go out as soon as its own P is ready, and one issuer's waits do not hold back
+        // the other's MMAs. Both walk the same pairs and K/V steps and release every K/V slot
+        // once (count 2 on the empty barriers): with a commit after using it, or with a plain
+        // arrive when their tile has no work in that step. The warp runs converged, so every
+        // descriptor and counter is warp-uniform; the elected lane (lane 0 of the full warp,
+        // always the same thread) issues each MMA and commit, so a commit covers all of them.
+        const int x = warp == 1 ? 0 : 1;
+        const uint32_t tS = tmem + x * 128, tO = tmem + 256 + x * 128;
         const uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
         const uint32_t idesc_pv = make_idesc_bf16(128, 128, 0, 1);
-        // descriptors of the first Q, K and V buffers; the others follow at fixed offsets
-        // (the start-address field is addr >> 4, and every buffer ends below 256 KB)
-        const uint64_t dq0 = make_sdesc_sw128(smem_u32(sQ), 16, 1024);
+        // descriptors of this tile's Q buffer and of the first K and V buffers; the other slots
+        // follow at fixed offsets (the start-address field is addr >> 4; all buffers end below 256 KB)
+        const uint64_t dq = make_sdesc_sw128(smem_u32(sQ + x * TC_Q_BYTES), 16, 1024);
         const uint64_t dk0 = make_sdesc_sw128(smem_u32(sK), 16, 1024);
         const uint64_t dv0 = make_sdesc_sw128(smem_u32(sV), 16384, 1024);
-        uint32_t gk = 0, gv = 0;                      // K / V steps consumed
-        uint32_t px0 = 0, px1 = 0, tx0 = 0, tx1 = 0;  // per tile: P V steps issued, tiles finished
+        uint32_t gk = 0, gv = 0;  // K / V steps consumed
+        uint32_t px = 0, tx = 0;  // P V steps issued, tiles finished
         bool ok = true;
         for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x) {
             const PairInfo pi = decode_pair(a, item);
             if (pi.ns == 0) continue;
-            const int64_t n0 = tile_steps(pi.t[0]), n1 = tile_steps(pi.t[1]);
+            const int64_t nx = tile_steps(x ? pi.t[1] : pi.t[0]);
             // completion #tx of q_full[x]: #tx-1 was waited for the previous tile of x
-            if (n0 > 0 && !(ok = tc_wait_warp(&bars->q_full[0], tx0 & 1, abort_flag))) break;
-            if (n1 > 0 && !(ok = tc_wait_warp(&bars->q_full[1], tx1 & 1, abort_flag))) break;
-            tc_fence_after();
+            if (nx > 0 && !(ok = tc_wait_warp(&bars->q_full[x], tx & 1, abort_flag))) break;
             for (int64_t i = 0; i <= pi.ns && ok; ++i) {
-                const bool do_qk = i < pi.ns;
-                const bool do_pv = i > 0;
+                const bool do_qk = i < pi.ns, do_pv = i > 0;
+                const bool my_qk = do_qk && i < nx, my_pv = do_pv && i - 1 < nx;
                 const uint32_t ks = gk % TC_KSLOTS, vs = gv % TC_VSLOTS;
-                const uint64_t kd = dk0 + (uint64_t)(ks * (TC_STEP_BYTES >> 4));
-                const uint64_t vd = dv0 + (uint64_t)(vs * (TC_STEP_BYTES >> 4));
+                // The K/V waits come first (those loads were issued long ago, P is the real gate).
+                // An issuer waits for every step's K and V even when its tile has no work in that
+                // step: its release of the slot below must not come before the slot was filled, or
+                // it would count toward the slot's previous use (completion #g/n - 1 of the empty
+                // barrier, which the producer waited for before this load).
                 if (do_pv && !(ok = tc_wait_warp(&bars->v_full[vs], (gv / TC_VSLOTS) & 1, abort_flag))) break;
-                bool k_ready = false;
-                // One tile's work of this iteration: P V for step i - 1, then Q K^T for step i.
-                auto tile = [&](const int x, const int64_t nx, uint32_t& pxx, uint32_t& txx) -> bool {
-                    const uint32_t tS = tmem + x * 128, tO = tmem + 256 + x * 128;
-                    if (do_pv && i - 1 < nx) {
-                        // completion #pxx of p_full[x]; #pxx-1 was waited before the previous P V of x
-                        if (!tc_wait_warp(&bars->p_full[x], pxx & 1, abort_flag)) return false;
-                        // O_x is free once the previous tile's epilogue has read it
-                        if (i == 1 && !tc_wait_warp(&bars->o_empty[x], (txx & 1) ^ 1, abort_flag)) return false;
-                        tc_fence_after();
-                        tc_mma_ts_w(tO, tS + 64, vd, idesc_pv, i > 1 ? 1u : 0u);
+                if (do_qk && !(ok = tc_wait_warp(&bars->k_full[ks], (gk / TC_KSLOTS) & 1, abort_flag))) break;
+                if (my_pv) {
+                    // completion #px of p_full[x]; #px-1 was waited before the previous P V
+                    if (!(ok = tc_wait_warp(&bars->p_full[x], px & 1, abort_flag))) break;
+                    // O_x is free once the previous tile's epilogue has read it
+                    if (i == 1 && !(ok = tc_wait_warp(&bars->o_empty[x], (tx & 1) ^ 1, abort_flag))) break;
+                }
+                tc_fence_after();
+                if (my_pv) {
+                    const uint64_t vd = dv0 + (uint64_t)(vs * (TC_STEP_BYTES >> 4));
+                    tc_mma_ts_w(tO, tS + 64, vd, idesc_pv, i > 1 ? 1u : 0u);
 #pragma unroll
-                        for (int k = 1; k < 8; ++k) tc_mma_ts_w(tO, tS + 64 + k * 8, vd + k * 128, idesc_pv, 1u);
-                        ++pxx;
-                        if (i == nx) {  // that was the tile's last step
-                            tc_commit_w(&bars->o_full[x]);
-                            ++txx;
-                        }
+                    for (int k = 1; k < 8; ++k) tc_mma_ts_w(tO, tS + 64 + k * 8, vd + k * 128, idesc_pv, 1u);
+                    ++px;
+                    if (i == nx) {  // that was the tile's last step
+                        tc_commit_w(&bars->o_full[x]);
+                        ++tx;
                     }
-                    if (do_qk && i < nx) {
-                        if (!k_ready) {
-                            if (!tc_wait_warp(&bars->k_full[ks], (gk / TC_KSLOTS) & 1, abort_flag)) return false;
-                            tc_fence_after();
-                            k_ready = true;
-                        }
-                        const uint64_t qd = dq0 + (uint64_t)(x * (TC_Q_BYTES >> 4));
+                }
+                if (my_qk) {
+                    const uint64_t kd = dk0 + (uint64_t)(ks * (TC_STEP_BYTES >> 4));
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
-                            tc_mma_ss_w(tS, qd + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
-                        }
-                        tc_commit_w(&bars->s_full[x]);
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+                        tc_mma_ss_w(tS, dq + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
                     }
-                    return true;
-                };
-                if (!(ok = tile(0, n0, px0, tx0))) break;
-                if (!(ok = tile(1, n1, px1, tx1))) break;
-                if (do_qk) {
-                    tc_commit_w(&bars->k_empty[ks]);  // both tiles' Q K^T of this step read K
+                    tc_commit_w(&bars->s_full[x]);
+                }
+                if (do_qk) {  // this issuer is done with K step gk
+                    if (my_qk) tc_commit_w(&bars->k_empty[ks]);
+                    else mbar_arrive_w(&bars->k_empty[ks]);
                     ++gk;
                 }
-                if (do_pv) {
-                    tc_commit_w(&bars->v_empty[vs]);  // both tiles' P V of the previous step read V
+                if (do_pv) {  // and with V step gv
+                    if (my_pv) tc_commit_w(&bars->v_empty[vs]);
+                    else mbar_arrive_w(&bars->v_empty[vs]);
                     ++gv;
                 }
             }
         }
-        // all MMAs issued by the elected lane have completed before TMEM is released
+        // all MMAs of this issuer have completed before TMEM is released
         __syncwarp();
-        tc_commit_w(&bars->final_mma);
-        mbar_wait(&bars->final_mma, 0);
+        tc_commit_w(&bars->final_mma[x]);
+        mbar_wait(&bars->final_mma[x], 0);
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax warps
