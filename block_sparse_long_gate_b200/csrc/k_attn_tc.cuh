@@ -64,6 +64,7 @@ struct TcBars {
     uint64_t o_full[2];   // per tile: the tile's last P V is in O_X
     uint64_t o_empty[2];  // per tile: the epilogue has read O_X
     uint64_t final_mma[2];  // per issuer: all of its MMAs have completed
+    uint64_t turn[2];       // issuer x may issue its MMAs of the current iteration
     uint32_t tmem_base;
     int abort_flag;
     uint32_t k_issued[TC_KSLOTS], v_issued[TC_VSLOTS];  // loads issued per slot (teardown bookkeeping)
@@ -265,8 +266,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         mbar_init(&bars->final_mma[0], 1);
         mbar_init(&bars->final_mma[1], 1);
+        mbar_init(&bars->turn[0], 1);
+        mbar_init(&bars->turn[1], 1);
         bars->abort_flag = 0;
         fence_mbarrier_init();
+        mbar_arrive(&bars->turn[0]);  // tile A's issuer goes first
     }
     if (warp == 1) {
         tmem_alloc(&bars->tmem_base, 512);
@@ -343,6 +347,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint64_t dv0 = make_sdesc_sw128(smem_u32(sV), 16384, 1024);
         uint32_t gk = 0, gv = 0;  // K / V steps consumed
         uint32_t px = 0, tx = 0;  // P V steps issued, tiles finished
+        uint32_t it = 0;          // iterations of the issue loop (the same sequence for both issuers)
         bool ok = true;
         for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x) {
             const PairInfo pi = decode_pair(a, item);
@@ -367,6 +372,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     // O_x is free once the previous tile's epilogue has read it
                     if (i == 1 && !(ok = tc_wait_warp(&bars->o_empty[x], (tx & 1) ^ 1, abort_flag))) break;
                 }
+                // Turns: the issuers alternate whole iterations (A, B, A, ...), so the tensor pipe
+                // runs one tile's batch before the other's and the two softmax groups stay out of
+                // phase (each softmax runs while the other tile's MMAs do). Completion #it of
+                // turn[x] is the other issuer's hand-over after its iteration it - 1 (for tile A's
+                // first iteration the initial arrival); #it-1 was waited at the previous iteration.
+                if (!(ok = tc_wait_warp(&bars->turn[x], it & 1, abort_flag))) break;
                 tc_fence_after();
                 if (my_pv) {
                     const uint64_t vd = dv0 + (uint64_t)(vs * (TC_STEP_BYTES >> 4));
@@ -388,6 +399,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     }
                     tc_commit_w(&bars->s_full[x]);
                 }
+                mbar_arrive_w(&bars->turn[x ^ 1]);
+                ++it;
                 if (do_qk) {  // this issuer is done with K step gk
                     if (my_qk) tc_commit_w(&bars->k_empty[ks]);
                     else mbar_arrive_w(&bars->k_empty[ks]);
