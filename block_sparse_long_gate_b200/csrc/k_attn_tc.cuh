@@ -366,18 +366,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 // barrier, which the producer waited for before this load).
                 if (do_pv && !(ok = tc_wait_warp(&bars->v_full[vs], (gv / TC_VSLOTS) & 1, abort_flag))) break;
                 if (do_qk && !(ok = tc_wait_warp(&bars->k_full[ks], (gk / TC_KSLOTS) & 1, abort_flag))) break;
-                if (my_pv) {
-                    // completion #px of p_full[x]; #px-1 was waited before the previous P V
-                    if (!(ok = tc_wait_warp(&bars->p_full[x], px & 1, abort_flag))) break;
-                    // O_x is free once the previous tile's epilogue has read it
-                    if (i == 1 && !(ok = tc_wait_warp(&bars->o_empty[x], (tx & 1) ^ 1, abort_flag))) break;
-                }
+                // O_x is free once the previous tile's epilogue has read it
+                if (my_pv && i == 1 && !(ok = tc_wait_warp(&bars->o_empty[x], (tx & 1) ^ 1, abort_flag))) break;
                 // Turns: the issuers alternate whole iterations (A, B, A, ...), so the tensor pipe
                 // runs one tile's batch before the other's and the two softmax groups stay out of
                 // phase (each softmax runs while the other tile's MMAs do). Completion #it of
                 // turn[x] is the other issuer's hand-over after its iteration it - 1 (for tile A's
                 // first iteration the initial arrival); #it-1 was waited at the previous iteration.
                 if (!(ok = tc_wait_warp(&bars->turn[x], it & 1, abort_flag))) break;
+                // P last: in steady state it is the event that gates the iteration.
+                // Completion #px of p_full[x]; #px-1 was waited before the previous P V.
+                if (my_pv && !(ok = tc_wait_warp(&bars->p_full[x], px & 1, abort_flag))) break;
                 tc_fence_after();
                 if (my_pv) {
                     const uint64_t vd = dv0 + (uint64_t)(vs * (TC_STEP_BYTES >> 4));
