@@ -158,7 +158,7 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
     return f2pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
                   __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
 }
-#define EXP2_POLY_PAIRS 3  // of every 8 pairs of a step, evaluated by exp2_poly2
+#define EXP2_POLY_PAIRS 2  // of every 8 pairs of a step, evaluated by exp2_poly2 (2 measured best of 1-4)
 
 // Masks the columns of a 64-key half (first column index c0) beyond `lim`.
 __device__ __forceinline__ void mask_cols(uint32_t (&sr)[2][32], int c0, int lim) {
