@@ -1,0 +1,93 @@
+"""GPU parity at the full sizes of the long-context workloads, in the launch path the
+benchmark times (moba_forward_ws with a caller workspace).
+
+The oracle cannot evaluate every row at these sizes, so each case checks a seeded sample
+of rows (every head, random tokens plus block edges) element by element against the fp64
+oracle, with the same selection / near-tie / tolerance rules as the small cases, and
+checks properties that hold at any size on every row:
+  - each selection row is well formed: ascending distinct earlier blocks, then the row's
+    own block, then -1 padding, with min(k, c + 1) entries;
+  - out and lse are finite everywhere.
+"""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from test_gpu_parity import _compare_outputs, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+LONG = [  # B, N, Hq, Hkv, block_size, topk, seed, sampled rows per head
+    (1, 131072, 32, 8, 4096, 12, 3, 24),     # Llama-3.1-8B attention shape at 128K
+    (1, 524288, 32, 8, 4096, 12, 3, 12),     # ... at 512K
+    (1, 1048576, 32, 8, 4096, 12, 3, 8),     # ... at 1M (the benchmark's workload)
+    (1, 10485760, 1, 1, 4096, 12, 4, 256),   # 10M tokens, one head
+]
+
+
+def _well_formed(idx, N, bs, topk):
+    """Device-side check of every selection row (see the module docstring)."""
+    B, H, n, k = idx.shape
+    t = torch.arange(n, device=idx.device, dtype=torch.int64)
+    c = (t // bs).view(1, 1, n)
+    cnt = torch.clamp(c + 1, max=topk)                        # entries a row must hold
+    valid = idx >= 0
+    assert torch.equal(valid.sum(-1), cnt.expand(B, H, n)), "entry count"
+    pos = torch.arange(k, device=idx.device).view(1, 1, 1, k)
+    assert bool((valid == (pos < cnt.unsqueeze(-1))).all()), "-1 padding only at the end"
+    last = idx.gather(-1, (cnt - 1).unsqueeze(-1).expand(B, H, n, 1)).squeeze(-1)
+    assert torch.equal(last.long(), c.expand(B, H, n)), "own block last"
+    inc = (idx[..., 1:] > idx[..., :-1]) | ~valid[..., 1:]
+    assert bool(inc.all()), "ascending distinct"
+
+
+@pytest.mark.parametrize("case", LONG, ids=lambda c: f"N{c[1]}_H{c[2]}")
+def test_long_context_sampled_rows(moba, cuda_dev, case):
+    B, N, Hq, Hkv, bs, topk, seed, per_head = case
+    gc.collect()
+    torch.cuda.empty_cache()  # blocks cached by earlier cases count as used in mem_get_info
+    free, _ = torch.cuda.mem_get_info(cuda_dev)
+    need = moba.workspace_size(B, Hq, Hkv, N, 128, bs, topk) + 3 * B * N * Hq * 128 * 2 + (4 << 30)
+    if free < need:
+        pytest.skip(f"needs {need / 2**30:.0f} GiB of device memory, {free / 2**30:.0f} GiB free")
+    q_h, k_h, v_h = synth.inputs(B, N, Hq, Hkv, 128, bs, seed)
+    q, k, v = q_h.to(cuda_dev), k_h.to(cuda_dev), v_h.to(cuda_dev)
+    ws = torch.empty(moba.workspace_size(B, Hq, Hkv, N, 128, bs, topk), dtype=torch.uint8, device=cuda_dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, N, dtype=torch.float32, device=cuda_dev)
+    moba.forward(q, k, v, bs, topk, out=out, lse=lse, workspace=ws)
+    idx = moba.gate(q, k, bs, topk)
+    assert moba.sync_status() == 0
+    _well_formed(idx, N, bs, topk)
+    assert bool(torch.isfinite(lse).all()) and bool(torch.isfinite(out).all())
+
+    rows = sample_rows(B, Hq, N, bs, topk, per_head, seed)
+    rt = torch.from_numpy(rows).to(cuda_dev)
+    gidx = idx[rt[:, 0], rt[:, 1], rt[:, 2]].cpu().numpy()
+    go = out[rt[:, 0], rt[:, 2], rt[:, 1]].float().cpu().numpy()
+    gl = lse[rt[:, 0], rt[:, 1], rt[:, 2]].cpu().numpy()
+    del ws
+    kbar = oracle.pool(k_h, bs)
+    sel, s_last, s_next = oracle.select(q_h, kbar, Hkv, bs, topk, rows)
+    ref_out, ref_lse = oracle.attend(q_h, k_h, v_h, bs, topk, rows, sel)
+
+    tie = oracle.near_tie(s_last, s_next)
+    mism = (gidx != sel).any(axis=1)
+    assert not (mism & ~tie).any(), f"{(mism & ~tie).sum()} selection mismatches outside near ties"
+    ok = ~mism
+    _compare_outputs(go[ok], gl[ok], ref_out[ok], ref_lse[ok], f"N={N}")
+    if mism.any():  # near ties: the oracle's selection injected for the whole tensor's affected rows
+        full = idx.clone()
+        full[rt[mism, 0], rt[mism, 1], rt[mism, 2]] = torch.from_numpy(sel[mism]).to(cuda_dev).to(full.dtype)
+        o2, l2 = moba.forward_selected(q, k, v, full, bs, topk)
+        assert moba.sync_status() == 0
+        go2 = o2[rt[:, 0], rt[:, 2], rt[:, 1]].float().cpu().numpy()
+        gl2 = l2[rt[:, 0], rt[:, 1], rt[:, 2]].cpu().numpy()
+        _compare_outputs(go2[mism], gl2[mism], ref_out[mism], ref_lse[mism], "injected")
+    del q, k, v, out, lse, idx
+    gc.collect()
+    torch.cuda.empty_cache()
