@@ -82,7 +82,8 @@ def test_long_context_sampled_rows(moba, cuda_dev, case):
     _compare_outputs(go[ok], gl[ok], ref_out[ok], ref_lse[ok], f"N={N}")
     if mism.any():  # near ties: the oracle's selection injected for the whole tensor's affected rows
         full = idx.clone()
-        full[rt[mism, 0], rt[mism, 1], rt[mism, 2]] = torch.from_numpy(sel[mism]).to(cuda_dev).to(full.dtype)
+        mt = rt[torch.from_numpy(mism).to(cuda_dev)]
+        full[mt[:, 0], mt[:, 1], mt[:, 2]] = torch.from_numpy(sel[mism]).to(cuda_dev).to(full.dtype)
         o2, l2 = moba.forward_selected(q, k, v, full, bs, topk)
         assert moba.sync_status() == 0
         go2 = o2[rt[:, 0], rt[:, 2], rt[:, 1]].float().cpu().numpy()
