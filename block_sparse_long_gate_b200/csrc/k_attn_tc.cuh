@@ -14,11 +14,13 @@
 // the softmax warps of A work on S_A, the MMAs of B run - and each K/V step in
 // shared memory feeds twice the MMA work.
 //
-// Roles (320 threads, one CTA per SM, persistent over the pairs):
+// Roles (352 threads, one CTA per SM, persistent over the pairs):
 //   warp 0     producer: TMA loads of K steps into a 3-slot ring and of V steps
 //              into a 2-slot ring (3-D maps, 128-byte swizzle); K runs one step ahead
-//   warp 1     MMA issuer (one thread) and TMEM owner. Per step i of a pair:
-//              [P V of A for step i-1, Q K^T of A for step i], then the same for B
+//   warp 1     MMA issuer of tile A (and TMEM owner), warp 10 MMA issuer of tile B.
+//              Per step i of a pair each issues [P V for step i-1, Q K^T for step i]
+//              of its tile; the two alternate whole iterations through turn barriers
+//              so the pipe runs one tile's batch, then the other's.
 //   warps 2-5  softmax of tile A; warps 6-9 softmax of tile B. Each thread owns one
 //              row: gathers its Q row (cp.async, swizzled), runs the softmax with a
 //              lazily moved maximum, and writes the normalised row in the epilogue.
@@ -35,7 +37,7 @@
 //
 // Every wait is bounded. A wait that reaches its limit records
 // MOBA_ERR_DEVICE_TIMEOUT and raises a CTA-wide abort flag; all roles then leave
-// their loops, the MMA thread waits (bounded) for its last MMAs, the producer
+// their loops, each MMA issuer waits (bounded) for its last MMAs, the producer
 // for its loads in flight, and the TMEM is freed before the CTA exits.
 #pragma once
 #include <cuda.h>
