@@ -192,41 +192,43 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, 2)
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = make_idesc_bf16(128, GATE_CAND, 0, 0);
-            uint32_t ti = 0, g = 0;
-            bool ok = true;
-            for (int64_t item = blockIdx.x; item < p.ntiles && ok; item += gridDim.x, ++ti) {
-                const GateTile gt = gate_tile(p, item);
-                if (!(ok = tc_wait(&bars->q_full, ti & 1, abort_flag))) break;
+        // The whole warp runs the loop, converged, and the elected lane (always lane 0)
+        // issues each MMA and commit: the operands stay warp-uniform, which keeps the issue
+        // rate when the top-k warps keep the SM sub-partition busy.
+        const uint32_t idesc = make_idesc_bf16(128, GATE_CAND, 0, 0);
+        const uint64_t dq = make_sdesc_sw128(smem_u32(sQ), 16, 1024);
+        const uint64_t dc0 = make_sdesc_sw128(smem_u32(sC), 16, 1024);
+        uint32_t ti = 0, g = 0;
+        bool ok = true;
+        for (int64_t item = blockIdx.x; item < p.ntiles && ok; item += gridDim.x, ++ti) {
+            const GateTile gt = gate_tile(p, item);
+            if (!(ok = tc_wait_warp(&bars->q_full, ti & 1, abort_flag))) break;
+            tc_fence_after();
+            for (int m = 0; m < gt.nch; ++m, ++g) {
+                const uint32_t s = g & 1;
+                if (!(ok = tc_wait_warp(&bars->c_full[s], (g >> 1) & 1, abort_flag))) break;
+                // the top-k threads have read this TMEM buffer two steps ago
+                if (!(ok = tc_wait_warp(&bars->s_empty[s], ((g >> 1) & 1) ^ 1, abort_flag))) break;
                 tc_fence_after();
-                const uint32_t sq = smem_u32(sQ);
-                for (int m = 0; m < gt.nch; ++m, ++g) {
-                    const uint32_t s = g & 1;
-                    if (!(ok = tc_wait(&bars->c_full[s], (g >> 1) & 1, abort_flag))) break;
-                    // the top-k threads have read this TMEM buffer two steps ago
-                    if (!(ok = tc_wait(&bars->s_empty[s], ((g >> 1) & 1) ^ 1, abort_flag))) break;
-                    tc_fence_after();
-                    const uint32_t sc = smem_u32(sC + s * GATE_STAGE_BYTES);
-                    const uint32_t tS = tmem + s * GATE_CAND;
+                const uint64_t dc = dc0 + (uint64_t)(s * (GATE_STAGE_BYTES >> 4));
+                const uint32_t tS = tmem + s * GATE_CAND;
 #pragma unroll
-                    for (int pl = 0; pl < 2; ++pl)
+                for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const uint32_t qoff = (k >> 2) * 16384 + (k & 3) * 32;
-                            const uint32_t coff = pl * 16384 + (k >> 2) * 8192 + (k & 3) * 32;
-                            tc_mma_ss(tS, make_sdesc_sw128(sq + qoff, 16, 1024),
-                                      make_sdesc_sw128(sc + coff, 16, 1024), idesc, (pl > 0 || k > 0) ? 1u : 0u);
-                        }
-                    tc_commit(&bars->c_empty[s]);
-                    tc_commit(&bars->s_full[s]);
-                }
-                if (!ok) break;
-                tc_commit(&bars->q_empty);  // the Q tile is no longer read by MMAs
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t qoff = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+                        const uint32_t coff = (pl * 16384 + (k >> 2) * 8192 + (k & 3) * 32) >> 4;
+                        tc_mma_ss_w(tS, dq + qoff, dc + coff, idesc, (pl > 0 || k > 0) ? 1u : 0u);
+                    }
+                tc_commit_w(&bars->c_empty[s]);
+                tc_commit_w(&bars->s_full[s]);
             }
-            tc_commit(&bars->final_mma);
-            mbar_wait(&bars->final_mma, 0);
+            if (!ok) break;
+            tc_commit_w(&bars->q_empty);  // the Q tile is no longer read by MMAs
         }
+        __syncwarp();
+        tc_commit_w(&bars->final_mma);
+        mbar_wait(&bars->final_mma, 0);
         __syncwarp();
     } else {
         // ------------------------------------------------------------ top-k threads
