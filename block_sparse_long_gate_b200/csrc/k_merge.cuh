@@ -29,15 +29,12 @@ __device__ __forceinline__ void fma8(float (&a)[8], float w, const uint4& x) {
     a[7] += w * bf16hi(x.w);
 }
 
-__global__ void __launch_bounds__(MERGE_THREADS) moba_merge_kernel(const int32_t* __restrict__ idx,
-                                                                   const uint16_t* __restrict__ opart,
-                                                                   const float* __restrict__ lpart, uint16_t* out,
-                                                                   float* lse, int64_t N, int Hq, int bs, int topk,
-                                                                   int64_t nrows) {
+// Merge of one row (b, hq, t) by one half-warp.
+__device__ __forceinline__ void merge_row(const int32_t* __restrict__ idx, const uint16_t* __restrict__ opart,
+                                          const float* __restrict__ lpart, uint16_t* out, float* lse, int64_t N,
+                                          int Hq, int bs, int topk, int64_t row) {
     const int lane = threadIdx.x & 15;  // lane within the half-warp
     const unsigned hmask = (threadIdx.x & 16) ? 0xFFFF0000u : 0x0000FFFFu;
-    const int64_t row = (int64_t)blockIdx.x * (MERGE_THREADS / 16) + (threadIdx.x >> 4);  // (b, hq, t)
-    if (row >= nrows) return;  // whole half-warps leave together
     const int64_t t = row % N;
     const int64_t bh = row / N;
     const int hq = (int)(bh % Hq);
@@ -109,4 +106,17 @@ __global__ void __launch_bounds__(MERGE_THREADS) moba_merge_kernel(const int32_t
     ow.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
     *reinterpret_cast<uint4*>(orow) = ow;
     if (lane == 0) lse[row] = L;
+}
+
+// Persistent: each half-warp walks the rows with a stride of all half-warps of the grid
+// (short-lived blocks of a row each left the SMs partly idle between block launches).
+__global__ void __launch_bounds__(MERGE_THREADS) moba_merge_kernel(const int32_t* __restrict__ idx,
+                                                                   const uint16_t* __restrict__ opart,
+                                                                   const float* __restrict__ lpart, uint16_t* out,
+                                                                   float* lse, int64_t N, int Hq, int bs, int topk,
+                                                                   int64_t nrows) {
+    const int64_t hw = (int64_t)blockIdx.x * (MERGE_THREADS / 16) + (threadIdx.x >> 4);
+    const int64_t stride = (int64_t)gridDim.x * (MERGE_THREADS / 16);
+    for (int64_t row = hw; row < nrows; row += stride)  // whole half-warps iterate together
+        merge_row(idx, opart, lpart, out, lse, N, Hq, bs, topk, row);
 }

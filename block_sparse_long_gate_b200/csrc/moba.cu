@@ -352,7 +352,15 @@ int run_attention(const Plan& P, const AttnParams& a, cudaStream_t st) {
 
 int run_merge(const Plan& P, const int32_t* idx, char* ws, void* out, float* lse, cudaStream_t st) {
     int64_t nrows = (int64_t)P.B * P.Hq * P.N;
-    moba_merge_kernel<<<(unsigned)cdiv(nrows, MERGE_THREADS / 16), MERGE_THREADS, 0, st>>>(
+    int dev = 0, nsm = 148, per_sm = 1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moba_merge_kernel, MERGE_THREADS, 0);
+    if (e != cudaSuccess) return cuda_fail(e);
+    int64_t grid = (int64_t)nsm * (per_sm > 0 ? per_sm : 1);
+    const int64_t need = cdiv(nrows, MERGE_THREADS / 16);
+    if (grid > need) grid = need;
+    moba_merge_kernel<<<(unsigned)grid, MERGE_THREADS, 0, st>>>(
         idx, (const uint16_t*)(ws + P.off_opart), (const float*)(ws + P.off_lpart), (uint16_t*)out, lse, P.N, P.Hq,
         P.bs, P.topk, nrows);
     count_launch();
