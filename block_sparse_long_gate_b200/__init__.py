@@ -31,7 +31,7 @@ EXPORTED = [
     "moba_status_string", "moba_workspace_size", "moba_forward", "moba_forward_ws", "moba_gate",
     "moba_forward_selected", "moba_forward_selected_ws", "moba_dense_causal", "moba_sync_status",
     "moba_set_attention_impl", "moba_set_gate_impl", "moba_stage_timing", "moba_stage_times",
-    "moba_launch_count", "moba_gate_noalloc", "moba_last_error_string",
+    "moba_launch_count", "moba_gate_noalloc", "moba_last_error_string", "moba_selftest_wait_timeout",
 ]
 STAGES = ("pool", "gate", "invert", "attention", "merge")
 
@@ -96,6 +96,8 @@ def lib():
             L.moba_launch_count.argtypes = []
             L.moba_last_error_string.restype = ctypes.c_char_p
             L.moba_last_error_string.argtypes = []
+            L.moba_selftest_wait_timeout.restype = _I
+            L.moba_selftest_wait_timeout.argtypes = [_L, _P]
             L.moba_gate_noalloc.restype = _I
             L.moba_gate_noalloc.argtypes = [_P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P]
             _lib = L
@@ -207,6 +209,12 @@ def dense_causal(q, k, v, out=None, lse=None, stream=None):
 def sync_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the library's device error flag."""
     return int(lib().moba_sync_status(_stream(stream)))
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Queue the bounded-wait self-test (a wait on a barrier nothing completes, given up
+    after limit_ns); the timeout shows up in the next sync_status()."""
+    _check(lib().moba_selftest_wait_timeout(int(limit_ns), _stream(stream)), "moba_selftest_wait_timeout")
 
 
 def check_status(stream=None):

@@ -205,9 +205,9 @@ __device__ __forceinline__ float softmax_half(const uint32_t (&sr)[2][32], uint3
 // Bounded wait that also gives up when another role raised the abort flag.
 // `backoff` adds a short sleep between polls (for roles off the critical path,
 // so their spinning does not take issue slots from the softmax warps).
-// The limit is wall-clock time (MOBA_WAIT_NS), read every 256 polls.
+// The limit is wall-clock time (limit_ns, MOBA_WAIT_NS by default), read every 256 polls.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                        bool backoff = false) {
+                                        bool backoff = false, uint64_t limit_ns = MOBA_WAIT_NS) {
     uint32_t n = 0;
     uint64_t t0 = 0;
     while (!mbar_try_wait(bar, parity)) {
@@ -216,7 +216,7 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
             const uint64_t now = global_ns();
             if (t0 == 0) {
                 t0 = now;
-            } else if (now - t0 > MOBA_WAIT_NS) {
+            } else if (now - t0 > limit_ns) {
                 moba_set_error(MOBA_ERR_DEVICE_TIMEOUT);
                 *abort_flag = 1;
                 return false;
@@ -225,6 +225,21 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
         if (backoff) __nanosleep(128);
     }
     return true;
+}
+
+// Failure-detection self-test: one warp waits, through tc_wait, on an mbarrier that
+// nothing ever completes. The wait must give up after limit_ns, record
+// MOBA_ERR_DEVICE_TIMEOUT and let the kernel return (no trap, no hang).
+__global__ void __launch_bounds__(32) moba_wait_selftest_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t never;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&never, 1);
+        abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    __syncwarp();
+    tc_wait(&never, 0, &abort_flag, false, limit_ns);
 }
 
 // Warp-uniform form for roles whose next instruction is a .sync.aligned tcgen05 op.

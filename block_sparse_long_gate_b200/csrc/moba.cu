@@ -525,6 +525,15 @@ int moba_sync_status(moba_stream_t stream) {
     return flag;
 }
 
+int moba_selftest_wait_timeout(int64_t limit_ns, moba_stream_t stream) {
+    if (limit_ns < 1000 || limit_ns > 10000000000LL) return MOBA_ERR_SHAPE;
+    int rc = check_device();
+    if (rc) return rc;
+    moba_wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_ns);
+    count_launch();
+    return launch_ok();
+}
+
 int moba_stage_timing(int enable) {
     std::lock_guard<std::mutex> lk(g_timing_mu);
     int old = g_timing ? 1 : 0;

@@ -30,8 +30,8 @@
  *     and runs asynchronously; an entry point returns once its work is queued.
  *   - Arguments are validated on the host before anything is queued; an invalid
  *     call returns a status code and queues nothing.
- *   - Asynchronous failures (a kernel wait that hit its iteration limit, a
- *     launch error) are reported by moba_sync_status().
+ *   - Asynchronous failures (a kernel wait that hit its limit, a launch error)
+ *     are reported by moba_sync_status().
  *   - Supported: d = 128, Hq % Hkv == 0, 1 <= topk <= 64, block_size >= 1,
  *     1 <= N, B * N < 2^31, ceil(N / block_size) <= 16384, B and Hq <= 65535, and a
  *     device of compute capability 10.0 (sm_100a).
@@ -128,6 +128,18 @@ int moba_dense_causal(const void* q, const void* k, const void* v, void* out, fl
  * MOBA_ERR_CUDA if the stream reported a CUDA error.
  */
 int moba_sync_status(moba_stream_t stream);
+
+/*
+ * Failure-detection self-test. Launches one warp on `stream` that waits, through the
+ * same bounded-wait routine the attention kernel uses, on an mbarrier that nothing
+ * ever completes, with a wall-clock limit of limit_ns. The wait gives up after the
+ * limit, records MOBA_ERR_DEVICE_TIMEOUT in the device error flag and the kernel
+ * returns, so moba_sync_status(stream) then reports MOBA_ERR_DEVICE_TIMEOUT and the
+ * context stays usable. Nothing faults, traps or hangs.
+ * Returns MOBA_ERR_SHAPE for limit_ns outside [1e3, 1e10], MOBA_ERR_UNSUPPORTED /
+ * MOBA_ERR_CUDA without a usable sm_100 device, MOBA_ERR_CUDA if the launch failed.
+ */
+int moba_selftest_wait_timeout(int64_t limit_ns, moba_stream_t stream);
 
 /*
  * Stage timing for measurement. While enabled, every moba_forward* call records

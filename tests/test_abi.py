@@ -78,3 +78,12 @@ def test_binding_refuses_cpu_tensors(moba):
     q = torch.zeros(1, 128, 1, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         moba.forward(q, q, q, 64, 2)
+
+
+def test_selftest_wait_timeout_checks_its_limit_on_host(moba):
+    L = moba.lib()
+    assert L.moba_selftest_wait_timeout(10, None) == 2            # below 1 us
+    assert L.moba_selftest_wait_timeout(10 ** 11, None) == 2      # above 10 s
+    import torch
+    if not torch.cuda.is_available():
+        assert L.moba_selftest_wait_timeout(10 ** 6, None) in (4, 5)  # no device: nothing runs
