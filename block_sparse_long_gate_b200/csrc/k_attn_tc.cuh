@@ -81,20 +81,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return r;
 }
 
-// Row maximum of 128 fp32 values held as 4 x 32 registers: four independent chains
-// of three-input maxima, so the reduction is throughput- rather than latency-bound.
-__device__ __forceinline__ float row_max128(const uint32_t (&v)[4][32]) {
-    float m[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        float a = max3f(__uint_as_float(v[c][0]), __uint_as_float(v[c][1]), __uint_as_float(v[c][2]));
-#pragma unroll
-        for (int j = 3; j + 1 < 32; j += 2) a = max3f(a, __uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1]));
-        m[c] = fmaxf(a, __uint_as_float(v[c][31]));
-    }
-    return max3f(m[0], m[1], fmaxf(m[2], m[3]));
-}
-
 __device__ __forceinline__ float row_max32(const uint32_t (&v)[32]) {
     float a0 = max3f(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
     float a1 = max3f(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5]));
