@@ -148,3 +148,15 @@ def test_malformed_selection_sets_error_flag(moba, cuda_dev):
     keep[200] = False
     assert torch.equal(lse[0, 0, keep], good_lse[0, 0, keep])
     assert moba.sync_status() == 0  # the flag was cleared
+
+
+@pytest.mark.parametrize("case", [(1, 1500, 4, 2, 200, 4), (2, 1000, 4, 2, 128, 3)])
+def test_cuda_core_attention_cross_check(moba, cuda_dev, case):
+    """The CUDA-core attention kernel, kept as an independent cross-check of the tensor-core
+    one, meets the same parity bar against the oracle."""
+    B, N, Hq, Hkv, bs, topk = case
+    old = moba.set_attention_impl(1)
+    try:
+        check_case(moba, cuda_dev, B, N, Hq, Hkv, bs, topk, 21)
+    finally:
+        moba.set_attention_impl(old)
