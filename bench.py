@@ -42,7 +42,8 @@ WORKLOAD_NAME = ("Llama-3.1-8B attention shape at 1M tokens: B=1, Hq=32, Hkv=8, 
 METRIC = "MoBA prefill fwd useful TFLOP/s @1M tokens"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-ATTN_SRC = os.path.join(ROOT, "block_sparse_long_gate_b200", "csrc", "k_attn_tc.cuh")
+ATTN_SRC = [os.path.join(ROOT, "block_sparse_long_gate_b200", "csrc", f)
+            for f in ("k_attn_tc.cuh", "k_attn_common.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
 
 
@@ -137,8 +138,11 @@ def attention_traffic() -> float | None:
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
-        with open(ATTN_SRC, "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
+        h = hashlib.sha256()
+        for path in ATTN_SRC:
+            with open(path, "rb") as f:
+                h.update(f.read())
+        digest = h.hexdigest()
         if rec.get("source_sha256") != digest:
             return None
         return float(rec["bytes_per_full_launch"])

@@ -32,6 +32,7 @@ struct AttnParams {
     const uint64_t* entries;
     const int64_t* segoff;      // list l spans entries [segoff[l*nch], segoff[(l+1)*nch])
     const int64_t* tile_start;  // past pair prefix per list, tile_start[L] = P
+    const int64_t* item_list;   // list of each past pair (find_list precomputed), [Pmax]
     int64_t L, Pmax;
     uint16_t* opart;  // bf16 [B, Hq, N, kp, d]
     float* lpart;     // fp32 [B, Hq, N, kp]
@@ -53,6 +54,15 @@ __device__ __forceinline__ int64_t find_list(const int64_t* __restrict__ ts, int
         else hi = mid;
     }
     return lo;
+}
+
+// item_list[p] = find_list(p) for every past pair p < P, -1 for p in [P, Pmax): the attention
+// roles then decode an item with one load instead of a binary search of dependent loads.
+__global__ void __launch_bounds__(256) moba_item_list_kernel(const int64_t* __restrict__ ts, int64_t L, int64_t Pmax,
+                                                             int64_t* __restrict__ item_list) {
+    const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (p >= Pmax) return;
+    item_list[p] = p < ts[L] ? find_list(ts, L, p) : -1;
 }
 
 struct TileInfo {
@@ -83,7 +93,7 @@ __device__ __forceinline__ PairInfo decode_pair(const AttnParams& a, int64_t ite
     if (item < a.Pmax) {
         const int64_t P = a.tile_start[a.L];
         if (item >= P) return pi;
-        const int64_t l = find_list(a.tile_start, a.L, item);
+        const int64_t l = a.item_list[item];
         const int64_t m = item - a.tile_start[l];
         const int64_t ls = a.segoff[l * a.nch], le = a.segoff[(l + 1) * a.nch];
         const int64_t j = l % a.nblk;

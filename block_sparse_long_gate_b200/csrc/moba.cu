@@ -79,7 +79,7 @@ struct Plan {
     int B, Hq, Hkv, G, d, bs, topk, kp;
     int64_t N, nblk, nfull, L, nch, E, Pmax, D, mb, ml, per_bh, nseg, nscan_parts;
     size_t off_kbar, off_planes, off_mu, off_stats, off_idx, off_counts, off_segoff, off_tiles, off_parts, off_entries,
-        off_opart, off_lpart, gate_bytes;
+        off_items, off_opart, off_lpart, gate_bytes;
     size_t total;
 };
 
@@ -143,6 +143,8 @@ int make_plan(int B, int Hq, int Hkv, int64_t N, int d, int bs, int topk, Plan* 
     o = align256(o + sizeof(int64_t) * (size_t)P.nscan_parts);
     P.off_entries = o;
     o = align256(o + sizeof(uint64_t) * (size_t)(P.E > 0 ? P.E : 1));
+    P.off_items = o;
+    o = align256(o + sizeof(int64_t) * (size_t)(P.Pmax > 0 ? P.Pmax : 1));
     P.off_opart = o;
     o = align256(o + sizeof(uint16_t) * (size_t)B * Hq * N * (P.kp > 0 ? P.kp : 1) * MOBA_D);
     P.off_lpart = o;
@@ -291,6 +293,12 @@ int run_invert(const Plan& P, const int32_t* idx, char* ws, cudaStream_t st) {
     if ((rc = run_scan(s1, P.nseg, parts, segoff, st))) return rc;
     ScanSrc s2{nullptr, segoff, P.nch};
     if ((rc = run_scan(s2, P.L, parts, tiles, st))) return rc;
+    if (P.Pmax > 0) {
+        moba_item_list_kernel<<<(unsigned)cdiv(P.Pmax, SCAN_THREADS), SCAN_THREADS, 0, st>>>(
+            tiles, P.L, P.Pmax, (int64_t*)(ws + P.off_items));
+        count_launch();
+        if ((rc = launch_ok())) return rc;
+    }
     moba_scatter_kernel<<<grid, INV_THREADS, sm_scatter, st>>>(idx, segoff, entries, P.N, P.Hq, P.Hkv, P.bs,
                                                                P.topk, P.nblk, P.nch);
     count_launch();
@@ -316,6 +324,7 @@ AttnParams attn_params(const Plan& P, const void* q, const void* k, const void* 
     a.entries = ws ? (const uint64_t*)(ws + P.off_entries) : nullptr;
     a.segoff = ws ? (const int64_t*)(ws + P.off_segoff) : nullptr;
     a.tile_start = ws ? (const int64_t*)(ws + P.off_tiles) : nullptr;
+    a.item_list = ws ? (const int64_t*)(ws + P.off_items) : nullptr;
     a.L = P.L;
     a.Pmax = P.Pmax;
     a.opart = ws ? (uint16_t*)(ws + P.off_opart) : nullptr;
