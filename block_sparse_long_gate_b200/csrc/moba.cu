@@ -155,12 +155,21 @@ int make_plan(int B, int Hq, int Hkv, int64_t N, int d, int bs, int topk, Plan* 
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
+// Records the text of a failed CUDA call for moba_last_error_string() and resets the
+// runtime's last-error state.
+int cuda_fail(cudaError_t e) {
+    g_last_cuda_error = cudaGetErrorString(e);
+    cudaGetLastError();
+    return MOBA_ERR_CUDA;
+}
+
 int check_device() {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MOBA_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
     int major = 0, minor = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MOBA_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return MOBA_ERR_CUDA;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) return cuda_fail(e);
     if (major != 10 || minor != 0) return MOBA_ERR_UNSUPPORTED;
     return MOBA_OK;
 }
@@ -178,11 +187,6 @@ int check_ptrs(std::initializer_list<const void*> ps) {
 void moba_note_cuda_error(cudaError_t e) { g_last_cuda_error = cudaGetErrorString(e); }
 
 namespace {
-
-int cuda_fail(cudaError_t e) {
-    g_last_cuda_error = cudaGetErrorString(e);
-    return MOBA_ERR_CUDA;
-}
 
 int launch_ok() {
     const cudaError_t e = cudaGetLastError();
@@ -210,9 +214,10 @@ bool use_tc_gate(const Plan& P) { return g_gate_impl == 0 && P.nfull > 0 && P.kp
 
 int run_pool(const Plan& P, const void* k, const GateScratch& gs, cudaStream_t st) {
     if (P.nfull == 0) return MOBA_OK;
-    if (gs.aux.head_stats &&
-        cudaMemsetAsync(gs.aux.head_stats, 0, sizeof(unsigned) * 2 * (size_t)P.B * P.Hkv, st) != cudaSuccess)
-        return MOBA_ERR_CUDA;
+    if (gs.aux.head_stats) {
+        const cudaError_t e = cudaMemsetAsync(gs.aux.head_stats, 0, sizeof(unsigned) * 2 * (size_t)P.B * P.Hkv, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
     dim3 grid((unsigned)P.nfull, P.Hkv, P.B);
     moba_pool_kernel<<<grid, POOL_THREADS, 0, st>>>((const uint16_t*)k, gs.kbar, P.N, P.Hkv, P.bs, P.nfull,
                                                     gs.aux);
@@ -279,11 +284,10 @@ int run_invert(const Plan& P, const int32_t* idx, char* ws, cudaStream_t st) {
     dim3 grid((unsigned)P.nch, P.Hkv, P.B);
     size_t sm_count = sizeof(uint32_t) * (size_t)P.nblk;
     size_t sm_scatter = (sizeof(int64_t) + sizeof(uint32_t)) * (size_t)P.nblk;
-    if (cudaFuncSetAttribute(moba_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_count) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(moba_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_scatter) !=
-            cudaSuccess)
-        return MOBA_ERR_CUDA;
+    cudaError_t e = cudaFuncSetAttribute(moba_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_count);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(moba_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_scatter);
+    if (e != cudaSuccess) return cuda_fail(e);
     moba_count_kernel<<<grid, INV_THREADS, sm_count, st>>>(idx, counts, P.N, P.Hq, P.Hkv, P.bs, P.topk, P.nblk,
                                                            P.nch);
     count_launch();
@@ -521,15 +525,13 @@ int moba_dense_causal(const void* q, const void* k, const void* v, void* out, fl
 }
 
 int moba_sync_status(moba_stream_t stream) {
-    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) {
-        cudaGetLastError();
-        return MOBA_ERR_CUDA;
-    }
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e);
     int flag = 0;
-    if (cudaMemcpyFromSymbol(&flag, g_moba_err, sizeof(int)) != cudaSuccess) return MOBA_ERR_CUDA;
+    if ((e = cudaMemcpyFromSymbol(&flag, g_moba_err, sizeof(int))) != cudaSuccess) return cuda_fail(e);
     if (flag) {
         int zero = 0;
-        if (cudaMemcpyToSymbol(g_moba_err, &zero, sizeof(int)) != cudaSuccess) return MOBA_ERR_CUDA;
+        if ((e = cudaMemcpyToSymbol(g_moba_err, &zero, sizeof(int))) != cudaSuccess) return cuda_fail(e);
     }
     return flag;
 }
