@@ -141,8 +141,19 @@ def forward(q, k, v, block_size: int, topk: int, rows: np.ndarray | None = None)
 
 
 def near_tie(s_last: np.ndarray, s_next: np.ndarray, rel: float = 1e-5) -> np.ndarray:
-    """Rows whose last selected and first unselected past scores differ by < rel (relative)."""
+    """Rows whose boundary is a near tie: the last selected and the first unselected past
+    scores differ by less than `rel` relative to the larger magnitude of the two,
+    |s_last - s_next| < rel * max(|s_last|, |s_next|). Equal scores (zero included) differ
+    by nothing and count as a tie. Rows without a boundary (every past block selected, so
+    both scores are NaN, or nothing selected by score, so s_last is NaN) are never ties.
+
+    This is the exemption rule of the selection check: only at such rows may another
+    implementation's selection differ from the oracle's, because the order of two
+    scores that close depends on rounding."""
+    s_last = np.asarray(s_last, dtype=np.float64)
+    s_next = np.asarray(s_next, dtype=np.float64)
     a = np.abs(s_last - s_next)
     m = np.maximum(np.abs(s_last), np.abs(s_next))
     with np.errstate(invalid="ignore"):
-        return np.nan_to_num(a < rel * m, nan=False).astype(bool)
+        tie = (a < rel * m) | (a == 0)
+    return tie & np.isfinite(s_last) & np.isfinite(s_next)
