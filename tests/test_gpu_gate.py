@@ -10,6 +10,7 @@ import pytest
 import torch
 
 import synth
+from parity_util import check_selection_all_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -37,15 +38,18 @@ def test_tc_gate_matches_fp64_gate(moba, cuda_dev, case):
     q, k, _ = synth.inputs(B, N, Hq, Hkv, 128, bs, seed)
     got, ref = _gates(moba, q.to(cuda_dev), k.to(cuda_dev), bs, topk)
     assert torch.equal(got, ref)
+    check_selection_all_rows(got, q, k, Hkv, bs, topk, f"gate case {case}")
 
 
 def test_tc_gate_crowded_scores(moba, cuda_dev):
-    """No block offsets: every block mean is small noise, scores crowd near the boundary."""
+    """No block offsets: every block mean is small noise, scores crowd near the boundary.
+    Both gates equal each other and the oracle's selection on every row."""
     B, N, Hq, Hkv, bs, topk = 1, 65536, 4, 1, 256, 16
     q = synth.normal(21, synth.Q_ID, (B, N, Hq, 128))
     k = synth.normal(21, synth.K_ID, (B, N, Hkv, 128))
     got, ref = _gates(moba, q.to(cuda_dev), k.to(cuda_dev), bs, topk)
     assert torch.equal(got, ref)
+    check_selection_all_rows(got, q, k, Hkv, bs, topk, "crowded scores")
 
 
 def test_tc_gate_exact_ties(moba, cuda_dev):
@@ -57,6 +61,10 @@ def test_tc_gate_exact_ties(moba, cuda_dev):
         k[:, j * bs:(j + 1) * bs] = k[:, (j - 5) * bs:(j - 4) * bs]
     got, ref = _gates(moba, q.to(cuda_dev), k.to(cuda_dev), bs, topk)
     assert torch.equal(got, ref)
-    # sanity: the duplicated pairs really produced ties that mattered somewhere
-    g = got.cpu().numpy()
-    assert g.shape == (B, Hq, N, topk)
+    # against the oracle on every row; exact ties are not excused: the lower index must win
+    check_selection_all_rows(got, q, k, Hkv, bs, topk, "exact ties", exact_ties_strict=True)
+    # the duplicated blocks really produced exact ties at the boundary of some rows
+    import oracle
+    rows = oracle.all_rows(B, Hq, N)
+    _, s_last, s_next = oracle.select(q, oracle.pool(k, bs), Hkv, bs, topk, rows)
+    assert int((s_last == s_next).sum()) > 100

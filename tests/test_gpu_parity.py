@@ -1,9 +1,10 @@
 """GPU parity: libmoba (through its C ABI) against the fp64 oracle on the same seeded inputs.
 
-Selections must match bit for bit, except at near ties: rows whose oracle
-(k-1)-th and k-th past scores differ by < 1e-5 relative. Those rows are
-re-checked with the oracle's selection injected. Outputs must be within
-max-abs 2e-2 and mean-abs 2e-3 (bf16 I/O) and lse within 1e-3.
+Selections are compared on EVERY row and must match bit for bit, except at near
+ties: rows whose oracle (k-1)-th and k-th past scores differ by < 1e-5 relative.
+Excused rows are counted, printed and bounded (at most 1e-4 of the rows), and
+re-checked with the oracle's selection injected. Outputs must be within max-abs
+2e-2 and mean-abs 2e-3 (bf16 I/O) and lse within 1e-3.
 """
 import numpy as np
 import pytest
@@ -11,10 +12,10 @@ import torch
 
 import oracle
 import synth
+from parity_util import (check_selection_all_rows, compare_outputs, gather_idx, gather_rows,
+                         sample_rows)
 
 pytestmark = pytest.mark.gpu
-
-OUT_MAX, OUT_MEAN, LSE_MAX = 2e-2, 2e-3, 1e-3
 
 
 def _inputs(B, N, Hq, Hkv, bs, seed, dev):
@@ -22,63 +23,33 @@ def _inputs(B, N, Hq, Hkv, bs, seed, dev):
     return (q, k, v), (q.to(dev), k.to(dev), v.to(dev))
 
 
-def sample_rows(B, Hq, N, bs, topk, per_head=256, seed=0):
-    """Seeded rows per (b, hq): random tokens plus block edges, the first and last block
-    and the rows with c <= k - 1."""
-    rng = np.random.default_rng(seed)
-    special = {0, N - 1, min(bs - 1, N - 1), min(bs, N - 1), min((topk - 1) * bs, N - 1),
-               min(topk * bs, N - 1), min(max(topk * bs - 1, 0), N - 1), N // 2}
-    rows = []
-    for b in range(B):
-        for h in range(Hq):
-            ts = set(rng.integers(0, N, size=min(per_head, N)).tolist()) | special
-            rows += [(b, h, t) for t in sorted(ts)]
-    return np.array(rows, dtype=np.int64)
-
-
-def _gather(gpu_out, gpu_lse, rows):
-    o = gpu_out.float().cpu().numpy()
-    l = gpu_lse.cpu().numpy()
-    return o[rows[:, 0], rows[:, 2], rows[:, 1]], l[rows[:, 0], rows[:, 1], rows[:, 2]]
-
-
-def _compare_outputs(out, lse, ref_out, ref_lse, what=""):
-    err = np.abs(out.astype(np.float64) - ref_out)
-    lerr = np.abs(lse.astype(np.float64) - ref_lse)
-    assert np.isfinite(out).all() and np.isfinite(lse).all(), what
-    assert err.max() <= OUT_MAX, (what, err.max())
-    assert err.mean() <= OUT_MEAN, (what, err.mean())
-    assert lerr.max() <= LSE_MAX, (what, lerr.max())
-    return err.max(), err.mean(), lerr.max()
-
-
 def check_case(moba, dev, B, N, Hq, Hkv, bs, topk, seed, rows=None):
+    """Selection of EVERY row against the oracle; outputs at `rows` (all rows by default)."""
     host, (q, k, v) = _inputs(B, N, Hq, Hkv, bs, seed, dev)
-    if rows is None:
-        rows = oracle.all_rows(B, Hq, N)
-    kbar = oracle.pool(host[1], bs)
-    sel, s_last, s_next = oracle.select(host[0], kbar, Hkv, bs, topk, rows)
-    ref_out, ref_lse = oracle.attend(*host, bs, topk, rows, sel)
-
     idx = moba.gate(q, k, bs, topk)
     out, lse = moba.forward(q, k, v, bs, topk)
     assert moba.sync_status() == 0
-    gidx = idx.cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
+    what = f"B={B} N={N} Hq={Hq} Hkv={Hkv} bs={bs} k={topk}"
+    rep = check_selection_all_rows(idx, host[0], host[1], Hkv, bs, topk, what)
 
-    tie = oracle.near_tie(s_last, s_next)
-    mism = (gidx != sel).any(axis=1)
-    assert not (mism & ~tie).any(), f"{(mism & ~tie).sum()} selection mismatches outside near ties"
-    go, gl = _gather(out, lse, rows)
+    if rows is None:
+        rows = oracle.all_rows(B, Hq, N)
+    kbar = oracle.pool(host[1], bs)
+    sel, _, _ = oracle.select(host[0], kbar, Hkv, bs, topk, rows)
+    ref_out, ref_lse = oracle.attend(*host, bs, topk, rows, sel)
+    mism = (gather_idx(idx, rows) != sel).any(axis=1)  # excused near ties (checked above)
+    go, gl = gather_rows(out, lse, rows)
     ok = ~mism
-    _compare_outputs(go[ok], gl[ok], ref_out[ok], ref_lse[ok], "forward")
+    compare_outputs(go[ok], gl[ok], ref_out[ok], ref_lse[ok], "forward")
     if mism.any():  # re-check the near-tie rows with the oracle's selection injected
         full = idx.clone()
-        full[rows[mism, 0], rows[mism, 1], rows[mism, 2]] = torch.from_numpy(sel[mism]).to(dev)
+        rt = torch.as_tensor(rows[mism], device=dev)
+        full[rt[:, 0], rt[:, 1], rt[:, 2]] = torch.from_numpy(sel[mism]).to(dev)
         o2, l2 = moba.forward_selected(q, k, v, full, bs, topk)
         assert moba.sync_status() == 0
-        go2, gl2 = _gather(o2, l2, rows)
-        _compare_outputs(go2[mism], gl2[mism], ref_out[mism], ref_lse[mism], "injected")
-    return {"rows": len(rows), "near_ties": int(tie.sum()), "mismatches": int(mism.sum())}
+        go2, gl2 = gather_rows(o2, l2, rows[mism])
+        compare_outputs(go2, gl2, ref_out[mism], ref_lse[mism], "injected")
+    return {"rows": rep.rows, "near_ties": rep.near_ties, "excused": rep.excused}
 
 
 SMALL = [  # B, N, Hq, Hkv, block_size, topk
@@ -102,15 +73,16 @@ def test_small_cases_all_rows(moba, cuda_dev, case):
 
 
 def test_single_head_long_sequence(moba, cuda_dev):
-    """Single head, N=32768, block 2048, top-3 (seed 1); sampled rows for the outputs."""
+    """Single head, N=32768, block 2048, top-3 (seed 1); selection on all rows, outputs on sampled rows."""
     B, N, Hq, Hkv, bs, topk = 1, 32768, 1, 1, 2048, 3
     check_case(moba, cuda_dev, B, N, Hq, Hkv, bs, topk, 1, rows=sample_rows(B, Hq, N, bs, topk, 2048))
 
 
 def test_fine_granularity_gqa(moba, cuda_dev):
-    """B=2, Hq=32, Hkv=8, N=32768, block 256, top-32 (seed 2); sampled rows."""
+    """B=2, Hq=32, Hkv=8, N=32768, block 256, top-32 (seed 2); selection on all 2.1M rows, outputs on
+    sampled rows."""
     B, N, Hq, Hkv, bs, topk = 2, 32768, 32, 8, 256, 32
-    check_case(moba, cuda_dev, B, N, Hq, Hkv, bs, topk, 2, rows=sample_rows(B, Hq, N, bs, topk, 48))
+    check_case(moba, cuda_dev, B, N, Hq, Hkv, bs, topk, 2, rows=sample_rows(B, Hq, N, bs, topk, 128))
 
 
 def test_dense_causal_matches_oracle(moba, cuda_dev):
@@ -121,8 +93,8 @@ def test_dense_causal_matches_oracle(moba, cuda_dev):
     r = oracle.forward(*host, 128, nblk, rows)
     out, lse = moba.dense_causal(q, k, v)
     assert moba.sync_status() == 0
-    go, gl = _gather(out, lse, rows)
-    _compare_outputs(go, gl, r["out"], r["lse"], "dense")
+    go, gl = gather_rows(out, lse, rows)
+    compare_outputs(go, gl, r["out"], r["lse"], "dense")
 
 
 def test_forward_is_deterministic(moba, cuda_dev):
