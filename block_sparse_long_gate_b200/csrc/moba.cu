@@ -28,8 +28,9 @@
 
 namespace {
 
-int g_attn_impl = 0;  // 0 tensor cores, 1 CUDA cores
-int g_gate_impl = 0;
+// Test hooks (process-wide): 0 = the default kernels, 1 = the CUDA-core cross-check kernels.
+std::atomic<int> g_attn_impl{0};  // attention: 0 tensor cores, 1 CUDA cores
+std::atomic<int> g_gate_impl{0};  // gate: 0 tensor cores + exact boundary, 1 CUDA-core fp64
 
 // Kernel launches made by the library (all devices, all threads).
 std::atomic<uint64_t> g_launches{0};
@@ -210,7 +211,7 @@ GateScratch gate_scratch(const Plan& P, char* ws, bool tc) {
     return g;
 }
 
-bool use_tc_gate(const Plan& P) { return g_gate_impl == 0 && P.nfull > 0 && P.kp > 0; }
+bool use_tc_gate(const Plan& P) { return g_gate_impl.load() == 0 && P.nfull > 0 && P.kp > 0; }
 
 int run_pool(const Plan& P, const void* k, const GateScratch& gs, cudaStream_t st) {
     if (P.nfull == 0) return MOBA_OK;
@@ -346,7 +347,7 @@ AttnParams attn_params(const Plan& P, const void* q, const void* k, const void* 
 
 int run_attention(const Plan& P, const AttnParams& a, cudaStream_t st) {
     const int64_t items = a.Pmax + a.D;
-    if (g_attn_impl == 1) {
+    if (g_attn_impl.load() == 1) {
         for (int64_t i0 = 0; i0 < items; i0 += (int64_t)1 << 30) {
             int64_t n = items - i0 < ((int64_t)1 << 30) ? items - i0 : ((int64_t)1 << 30);
             moba_attn_simt_kernel<<<(unsigned)n, 128, 0, st>>>(a, i0);
@@ -579,15 +580,13 @@ uint64_t moba_launch_count(void) { return g_launches.load(); }
 const char* moba_last_error_string(void) { return g_last_cuda_error; }
 
 int moba_set_attention_impl(int impl) {
-    int old = g_attn_impl;
-    g_attn_impl = impl;
-    return old;
+    if (impl != 0 && impl != 1) return MOBA_ERR_SHAPE;
+    return g_attn_impl.exchange(impl);
 }
 
 int moba_set_gate_impl(int impl) {
-    int old = g_gate_impl;
-    g_gate_impl = impl;
-    return old;
+    if (impl != 0 && impl != 1) return MOBA_ERR_SHAPE;
+    return g_gate_impl.exchange(impl);
 }
 
 }  // extern "C"
@@ -597,25 +596,61 @@ int moba_set_gate_impl(int impl) {
 // that reserve nearly all HBM up front for their KV cache and hand out only
 // pre-planned buffers (a cudaMallocAsync there either fails or breaks the plan),
 // and embedders with a fixed, audited memory budget that forbids allocation
-// inside a call. moba_gate_noalloc serves them: it runs the same pooling and gate
-// kernels as moba_gate, but the gate's only scratch, the fp64 block means, lives
-// in the fixed array below instead of a stream-ordered allocation.
+// inside a call. moba_gate_noalloc serves them: it runs the pooling kernel and
+// the fp64 CUDA-core gate (the gate whose only scratch is the block means), and
+// those block means live in the fixed array below instead of a stream-ordered
+// allocation. Its selections are the ones moba_gate returns (both gates give
+// the exact fp64 selection); at long sequences it is slower than moba_gate's
+// default tensor-core gate.
 //
 // The array is part of the library image: every GPU that loads the library holds
 // its 8 MiB until the process exits. In host code its name is only a host-side
-// stand-in, so the device address is looked up with cudaGetSymbolAddress, once
-// per device, on the first call made with that device current (that first call
-// should therefore come before any stream capture). All calls share the array
-// and it keeps the last call's contents; the pooling kernel overwrites every
-// entry the gate reads, so nothing needs clearing. Calls that overlap on the GPU
-// (different streams, or different host threads, on the same device) race on it.
+// stand-in, so the device address is looked up with cudaGetSymbolAddress on the
+// first call made with a device current (that first call should therefore come
+// before any stream capture), and looked up again only when the calling thread's
+// CUDA context is a different one than at the last lookup on that device (after a
+// device reset, the module is loaded again at another address). All calls share
+// the array and it keeps the last call's contents; the pooling kernel overwrites
+// every entry the gate reads, so nothing needs clearing. Calls that overlap on the
+// GPU (different streams, or different host threads, on the same device) race on it.
 #define MOBA_NOALLOC_KBAR_ROWS 8192  // B * Hkv * floor(N / block_size) <= 8192 (8 MiB of doubles)
 static __device__ __align__(256) double g_noalloc_kbar[MOBA_NOALLOC_KBAR_ROWS * MOBA_D];
 
 namespace {
 std::mutex g_noalloc_mu;
 constexpr int kNoallocMaxDevices = 64;
-double* g_noalloc_dev_ptr[kNoallocMaxDevices] = {};
+struct NoallocSlot {
+    double* ptr;
+    unsigned long long ctx_id;
+    bool have_id;
+};
+NoallocSlot g_noalloc_slot[kNoallocMaxDevices] = {};
+
+typedef CUresult (*moba_ctx_get_current_fn)(CUcontext*);
+typedef CUresult (*moba_ctx_get_id_fn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context (false when there is none yet,
+// or when the driver does not offer the query).
+bool current_ctx_id(unsigned long long* id) {
+    static moba_ctx_get_current_fn get_cur = nullptr;
+    static moba_ctx_get_id_fn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_cur = (moba_ctx_get_current_fn)p;
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = (moba_ctx_get_id_fn)p;
+    });
+    if (!get_cur || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
 }  // namespace
 
 extern "C" int moba_gate_noalloc(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv, int64_t N,
@@ -627,20 +662,23 @@ extern "C" int moba_gate_noalloc(const void* q, const void* k, int32_t* idx, int
     if ((rc = check_ptrs({q, k, (const void*)idx}))) return rc;
     if ((rc = check_device())) return rc;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MOBA_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
     if (dev < 0 || dev >= kNoallocMaxDevices) return MOBA_ERR_UNSUPPORTED;
     double* kbar = nullptr;
     {
         std::lock_guard<std::mutex> lk(g_noalloc_mu);
-        if (!g_noalloc_dev_ptr[dev]) {
+        NoallocSlot& slot = g_noalloc_slot[dev];
+        unsigned long long ctx = 0;
+        const bool have = current_ctx_id(&ctx);
+        if (!slot.ptr || !have || !slot.have_id || slot.ctx_id != ctx) {
             void* p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_noalloc_kbar) != cudaSuccess || !p) {
-                cudaGetLastError();
-                return MOBA_ERR_CUDA;
-            }
-            g_noalloc_dev_ptr[dev] = (double*)p;
+            if ((e = cudaGetSymbolAddress(&p, g_noalloc_kbar)) != cudaSuccess) return cuda_fail(e);
+            if (!p) return MOBA_ERR_CUDA;
+            slot.ptr = (double*)p;
+            slot.have_id = current_ctx_id(&slot.ctx_id);  // the lookup made the context current
         }
-        kbar = g_noalloc_dev_ptr[dev];
+        kbar = slot.ptr;
     }
     cudaStream_t st = (cudaStream_t)stream;
     GateScratch gs;

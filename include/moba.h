@@ -76,6 +76,11 @@ int moba_workspace_size(int B, int Hq, int Hkv, int64_t N, int d, int block_size
 /*
  * The whole causal prefill forward: pooling, gating, top-k with the forced own
  * block, selection inversion, block-sparse attention and log-sum-exp merge.
+ * Defined by: "MoBA project hub" page, Steps 1-3 (partition, parameter-less
+ * gating, attention over the kept blocks merged by log-sum-exp); "MoBA
+ * tech-report summary" page, section 2 (block partition, score s_i and top-k,
+ * causality: no future block, own block always kept and masked causally);
+ * "NSA vs MoBA" blog, section 1 (softmax(q k^T / sqrt(d)) v).
  * Writes out and lse. Allocates its workspace with cudaMallocAsync on `stream`
  * and frees it on the same stream.
  */
@@ -92,6 +97,11 @@ int moba_forward_ws(const void* q, const void* k, const void* v, void* out, floa
 /*
  * Gating only: block mean pooling, scores <q_t, Kbar_j> over earlier blocks,
  * forced own block and top-k. Writes idx (int32 [B, Hq, N, topk]).
+ * Defined by: "MoBA project hub" page, Step 2 (score of a block = inner product
+ * of the query with the block's mean-pooled keys, no gate parameters, top-k);
+ * "KIMI MoBA" blog, section 3 (score_pooling = mean, causal_mask,
+ * current_block_force); "MoBA tech-report summary" page, section 2 (score s_i,
+ * top-k, causality). Ties at the boundary go to the lower block index.
  * Allocates its small scratch (the block means) with cudaMallocAsync on `stream`.
  */
 int moba_gate(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv, int64_t N, int d,
@@ -99,7 +109,11 @@ int moba_gate(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv
 
 /*
  * Attention with a given selection idx (same layout as moba_gate's output):
- * selection inversion, block-sparse attention and merge. Each row must list
+ * selection inversion, block-sparse attention and merge. Defined by: "MoBA
+ * project hub" page, Step 3 (attention over the selected blocks, the own block
+ * masked causally, partial results fused by log-sum-exp); "MoBA tech-report
+ * summary" page, section 2, implementation steps 1-5 (queries grouped per key
+ * block, attention per block, outputs combined by online softmax). Each row must list
  * distinct blocks <= c(t) and include c(t); a malformed row is skipped and
  * reported as MOBA_ERR_SELECTION by moba_sync_status(). Allocates its
  * workspace with cudaMallocAsync on `stream`.
@@ -160,12 +174,16 @@ int moba_stage_times(float* ms, int n, int* calls);
  * moba_gate without any device allocation, for callers that cannot allocate
  * while they run (serving engines that pre-plan every byte of HBM for their KV
  * cache, embedders with a fixed memory budget). The MoBA pages have no
- * counterpart: this is a library convenience. Same arguments, results and
- * kernels as moba_gate; its scratch (the block means) is a fixed 8 MiB device
- * array inside the library, held by every GPU that loads it until exit.
+ * counterpart: this is a library convenience. Same arguments and results as
+ * moba_gate. It always runs the fp64 CUDA-core gate (whose only scratch is the
+ * block means), so its selections are moba_gate's, but at long sequences it is
+ * slower than moba_gate's default tensor-core gate. Its scratch is a fixed
+ * 8 MiB device array inside the library, held by every GPU that loads it until exit.
  *   - Limit: B * Hkv * floor(N / block_size) <= 8192, else MOBA_ERR_SHAPE.
  *   - The first call on a device looks up the array's device address with that
- *     device current; make that first call before any stream capture.
+ *     device current; make that first call before any stream capture. The
+ *     address is looked up again when the current CUDA context changed since
+ *     (for example after a device reset).
  *   - All calls share the array: calls that overlap on the GPU race on it.
  *     Nothing in it needs clearing (each call overwrites what it reads).
  */
@@ -179,12 +197,18 @@ const char* moba_last_error_string(void);
 /* Number of kernels the library has launched in this process (all devices). */
 uint64_t moba_launch_count(void);
 
-/* Implementation selector for the attention step: 0 = tensor-core kernel (default),
- * 1 = the simple CUDA-core kernel kept as a cross-check. Returns the previous value. */
+/* TEST HOOK, process-wide. Implementation of the attention step used by every later call
+ * from any thread of the process: 0 = tensor-core kernel (default), 1 = the simple
+ * CUDA-core kernel kept only as an independent cross-check in the tests. Values other
+ * than 0 and 1 are refused (MOBA_ERR_SHAPE is returned and nothing changes); otherwise
+ * returns the previous value. The switch is atomic, but calls that run while another
+ * thread changes it may use either kernel: set it once, before any concurrent use. */
 int moba_set_attention_impl(int impl);
 
-/* Implementation selector for the gate: 0 = default, 1 = the CUDA-core fp64 kernel.
- * Returns the previous value. */
+/* TEST HOOK, process-wide, same rules as moba_set_attention_impl: the gate used by every
+ * later call, 0 = default (tensor-core gate with exact fp64 boundary re-scoring), 1 = the
+ * CUDA-core fp64 gate kept as a cross-check. Returns the previous value, or MOBA_ERR_SHAPE
+ * for any other value. */
 int moba_set_gate_impl(int impl);
 
 #ifdef __cplusplus

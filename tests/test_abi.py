@@ -87,3 +87,9 @@ def test_selftest_wait_timeout_checks_its_limit_on_host(moba):
     import torch
     if not torch.cuda.is_available():
         assert L.moba_selftest_wait_timeout(10 ** 6, None) in (4, 5)  # no device: nothing runs
+
+
+def test_test_hooks_refuse_unknown_values(moba):
+    L = moba.lib()
+    assert L.moba_set_attention_impl(7) == 2 and L.moba_set_gate_impl(-1) == 2
+    assert L.moba_set_attention_impl(0) == 0 and L.moba_set_gate_impl(0) == 0  # previous values
