@@ -2,24 +2,30 @@
 """Benchmark of the MoBA causal prefill forward on B200.
 
 Workload (one step = one whole forward: pooling, gating + top-k, selection
-inversion, block-sparse attention, log-sum-exp merge): the Llama-3.1-8B
-attention shape at one million tokens, B=1, Hq=32, Hkv=8, d=128,
+inversion, block-sparse attention, log-sum-exp merge), by default the
+Llama-3.1-8B attention shape at one million tokens: B=1, Hq=32, Hkv=8, d=128,
 N=1048576, block_size=4096, topk=12, bf16, seeded synthetic inputs with the
 pages' distribution (Q, V ~ N(0,1); K = N(0,1) + a per key-block offset
-N(0, 0.5^2)), seed 3.
+N(0, 0.5^2)), seed 3. `--config` selects the other workloads of the same
+family (0: tiny single head, 1: single head at 32K, 2: fine-granularity GQA,
+3: the Llama shape, with `--seq-len` for 128K / 512K, 4: 10M tokens, one head).
 
 Metric: useful TFLOP/s (4 d FLOPs per attended query/key pair) and ms per
 forward; the JSON line also carries the fraction of the bf16 tensor-core peak,
-the speedup over dense causal attention on the same GPU, the end-to-end number
-through host buffers, the attention kernel's roofline and the CPU oracle
-baseline.
+the speedup over dense causal attention on the same GPU (this library's dense
+kernel and torch's scaled_dot_product_attention, the faster of the two), the
+end-to-end number through host buffers, the attention kernel's roofline and the
+CPU oracle baseline.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl moba|reference]
+  python bench.py [--config C] [--gpus N] [--steps K] [--warmup W] [--impl moba|reference]
 
-With N > 1 (one process per GPU under torch.distributed.run) every rank runs
-its own independent forward of the same shape (weak scaling; the method has no
-exchange step between sequences). `--impl reference` times the fp64 CPU oracle
-on a bounded sample of the same workload on the host cores.
+With N > 1 (one process per GPU under torch.distributed.run) one forward is split
+by kv-head groups: rank r owns a contiguous range of kv heads and their query
+heads, and runs the single-GPU forward on its slices with no exchange between
+ranks (total work fixed: strong scaling). Workloads with fewer kv heads than
+ranks run one independent forward per rank instead (weak scaling).
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload on the host cores.
 """
 from __future__ import annotations
 
@@ -36,36 +42,58 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = {"B": 1, "Hq": 32, "Hkv": 8, "d": 128, "N": 1 << 20, "block_size": 4096, "topk": 12, "seed": 3}
+CONFIGS = {
+    0: {"B": 1, "Hq": 1, "Hkv": 1, "d": 128, "N": 4096, "block_size": 512, "topk": 3, "seed": 0},
+    1: {"B": 1, "Hq": 1, "Hkv": 1, "d": 128, "N": 32768, "block_size": 2048, "topk": 3, "seed": 1},
+    2: {"B": 2, "Hq": 32, "Hkv": 8, "d": 128, "N": 32768, "block_size": 256, "topk": 32, "seed": 2},
+    3: {"B": 1, "Hq": 32, "Hkv": 8, "d": 128, "N": 1 << 20, "block_size": 4096, "topk": 12, "seed": 3},
+    4: {"B": 1, "Hq": 1, "Hkv": 1, "d": 128, "N": 10485760, "block_size": 4096, "topk": 12, "seed": 4},
+}
+CONFIG_NAMES = {
+    0: "Tiny reference",
+    1: "Single-head long sequence",
+    2: "Fine-granularity GQA",
+    3: "Llama-3.1-8B attention shape at long context",
+    4: "Extreme length (10M tokens, one head)",
+}
+DEFAULT_CONFIG = 3
+WORKLOAD = CONFIGS[DEFAULT_CONFIG]
 WORKLOAD_NAME = ("Llama-3.1-8B attention shape at 1M tokens: B=1, Hq=32, Hkv=8, d=128, N=1048576, "
                  "block_size=4096, topk=12, causal, bf16, seed 3")
 METRIC = "MoBA prefill fwd useful TFLOP/s @1M tokens"
 UNIT = "TFLOP/s"
+SPEC_BF16_TFLOPS = 2250.0  # nominal dense bf16 tensor-core peak of one B200, for context
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ATTN_SRC = [os.path.join(ROOT, "block_sparse_long_gate_b200", "csrc", f)
             for f in ("k_attn_tc.cuh", "k_attn_common.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
+L2_FLUSH_BELOW = 512 << 20  # inputs smaller than this get an L2 flush between timed steps
 
 
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--config", type=int, choices=sorted(CONFIGS), default=DEFAULT_CONFIG)
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=5)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=("moba", "reference"), default="moba")
-    p.add_argument("--seq-len", type=int, default=WORKLOAD["N"], help="override N (diagnostic runs only)")
+    p.add_argument("--seq-len", type=int, default=None,
+                   help="override N (config 3: 131072 / 524288 / 1048576; other values are diagnostic)")
     p.add_argument("--hq", type=int, default=None, help="override Hq (diagnostic runs only)")
     p.add_argument("--hkv", type=int, default=None, help="override Hkv (diagnostic runs only)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-dense", action="store_true")
+    p.add_argument("--no-sdpa", action="store_true", help="skip torch's dense attention in the dense arm")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--sample-rows", type=int, default=1024, help="oracle rows per CPU sample")
     return p.parse_args(argv)
 
 
 # ---------------------------------------------------------------- helpers shared with the tests
-def workload(seq_len: int | None = None, hq: int | None = None, hkv: int | None = None) -> dict:
-    w = dict(WORKLOAD)
+def workload(seq_len: int | None = None, hq: int | None = None, hkv: int | None = None,
+             config: int = DEFAULT_CONFIG) -> dict:
+    w = dict(CONFIGS[config])
+    w["config"] = config
     if seq_len:
         w["N"] = int(seq_len)
     if hq:
@@ -76,9 +104,22 @@ def workload(seq_len: int | None = None, hq: int | None = None, hkv: int | None 
 
 
 def workload_name(w: dict) -> str:
-    if all(w[k] == WORKLOAD[k] for k in ("N", "Hq", "Hkv")):
+    cfg = w.get("config", DEFAULT_CONFIG)
+    base = CONFIGS[cfg]
+    if cfg == DEFAULT_CONFIG and all(w[k] == WORKLOAD[k] for k in ("N", "Hq", "Hkv")):
         return WORKLOAD_NAME
-    return f"{WORKLOAD_NAME} (diagnostic override: N={w['N']}, Hq={w['Hq']}, Hkv={w['Hkv']})"
+    name = (f"{CONFIG_NAMES[cfg]}: B={w['B']}, Hq={w['Hq']}, Hkv={w['Hkv']}, d={w['d']}, N={w['N']}, "
+            f"block_size={w['block_size']}, topk={w['topk']}, causal, bf16, seed {w['seed']}")
+    if any(w[k] != base[k] for k in ("Hq", "Hkv")) or (w["N"] != base["N"] and not (
+            cfg == 3 and w["N"] in (131072, 524288))):
+        name += " (diagnostic override)"
+    return name
+
+
+def metric_name(w: dict) -> str:
+    if w.get("config", DEFAULT_CONFIG) == DEFAULT_CONFIG and w["N"] == WORKLOAD["N"]:
+        return METRIC
+    return f"MoBA prefill fwd useful TFLOP/s @{w['N']} tokens"
 
 
 def useful_flops(w: dict) -> float:
@@ -209,18 +250,31 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle baseline
 def oracle_sample(q, k, v, w: dict, n_rows: int, seed: int) -> tuple[float, float, int]:
-    """Time the oracle on a row sample: (seconds, useful FLOPs of the sample, rows)."""
+    """Time the oracle on a row sample (every row when the workload has no more than n_rows):
+    (seconds, useful FLOPs of the sample, rows)."""
     import oracle
-    rows = sample_rows(w, n_rows, seed)
+    total = w["B"] * w["Hq"] * w["N"]
+    rows = oracle.all_rows(w["B"], w["Hq"], w["N"]) if total <= n_rows else sample_rows(w, n_rows, seed)
     t0 = time.perf_counter()
     oracle.forward(q, k, v, w["block_size"], w["topk"], rows)
     dt = time.perf_counter() - t0
     return dt, rows_useful_flops(w, rows), len(rows)
 
 
-def host_inputs(w: dict, seed: int, pin: bool):
+def sample_text(w: dict, nrows: int) -> str:
+    total = w["B"] * w["Hq"] * w["N"]
+    if nrows >= total:
+        return f"all {total} rows of the workload per step (pool, gate and attention in fp64)"
+    return (f"{nrows} seeded rows per step spread over all {w['B'] * w['Hq']} heads and the whole sequence; "
+            f"each step pools all of K, then gates and attends the sampled rows in fp64")
+
+
+def host_inputs(w: dict, seed: int, pin: bool, hkv_range=None):
     import synth
-    return synth.inputs(w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], w["block_size"], seed, pin=pin)
+    if hkv_range is None:
+        return synth.inputs(w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], w["block_size"], seed, pin=pin)
+    return synth.inputs_heads(w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], w["block_size"], seed,
+                              hkv_range[0], hkv_range[1], pin=pin)
 
 
 def cpu_cores() -> int:
@@ -228,34 +282,99 @@ def cpu_cores() -> int:
     return int(n) if n and n.isdigit() else (os.cpu_count() or 1)
 
 
+def peak_fields(value_per_gpu: float, clocks: dict, peaks: dict, peak_src: str) -> dict:
+    """Fractions of the bf16 tensor-core peak: the measured burst cuBLAS figure (headline),
+    the measured sustained one, the nominal spec, and the burst fraction at the SM clock
+    the run saw scaled to the maximum clock (so the power cap's share is visible)."""
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    out = {
+        "pct_of_peak": 100.0 * value_per_gpu / burst,
+        "peak_tflops": burst,
+        "peak_source": f"bf16_tflops (burst cuBLAS bf16 GEMM) of {peak_src}",
+        "pct_of_sustained_peak": 100.0 * value_per_gpu / sust,
+        "sustained_peak_tflops": sust,
+        "pct_of_spec_peak": 100.0 * value_per_gpu / SPEC_BF16_TFLOPS,
+        "spec_peak_tflops": SPEC_BF16_TFLOPS,
+    }
+    sm, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if sm and mx:
+        out["clock_normalised_tflops"] = value_per_gpu * mx / sm
+        out["pct_of_peak_at_max_clock"] = 100.0 * value_per_gpu * mx / sm / burst
+    return out
+
+
 # ---------------------------------------------------------------- reference arm (the oracle)
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    w = workload(args.seq_len, args.hq, args.hkv)
+    w = workload(args.seq_len, args.hq, args.hkv, args.config)
     q, k, v = host_inputs(w, w["seed"], pin=False)
     for i in range(args.warmup):
         oracle_sample(q, k, v, w, args.sample_rows, 1000 + i)
     secs, fl = 0.0, 0.0
+    nrows = 0
     for i in range(args.steps):
         dt, f, nrows = oracle_sample(q, k, v, w, args.sample_rows, 2000 + i)
         secs += dt
         fl += f
     value = fl / secs / 1e12
-    sample = (f"{nrows} seeded rows per step spread over all {w['B'] * w['Hq']} heads and the whole sequence; "
-              f"each step pools all of K, then gates and attends the sampled rows in fp64")
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric_name(w), "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_name(w),
                    "global_batch": w["B"], "seq_len": w["N"], "parallelism": "host cores (OpenMP)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": sample_text(w, nrows)},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ---------------------------------------------------------------- dense comparison
+def time_sdpa(q, k, v, stream) -> dict:
+    """torch's scaled_dot_product_attention, causal, with its fused backends only (no math
+    fallback, which would materialise N x N): grouped-query heads through enable_gqa, or with
+    the kv heads repeated (outside the timed region) when no fused backend takes enable_gqa."""
+    import torch
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    F = torch.nn.functional
+    backends = [SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION]
+    G = q.shape[2] // k.shape[2]
+    qt, kt, vt = q.transpose(1, 2), k.transpose(1, 2), v.transpose(1, 2)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+
+    def attempt(kk, vv, gqa):
+        with sdpa_kernel(backends):
+            F.scaled_dot_product_attention(qt[:, :, :4096], kk[:, :, :4096], vv[:, :, :4096], is_causal=True,
+                                           enable_gqa=gqa)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            o = F.scaled_dot_product_attention(qt, kk, vv, is_causal=True, enable_gqa=gqa)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        del o
+        return e0.elapsed_time(e1)
+
+    try:
+        return {"ms": attempt(kt, vt, G > 1), "kernel": "torch sdpa" + (" (enable_gqa)" if G > 1 else "")}
+    except RuntimeError as exc:
+        if G == 1:
+            return {"error": str(exc).splitlines()[0][:200]}
+        first = str(exc).splitlines()[0][:120]
+    torch.cuda.empty_cache()
+    try:
+        kr = kt.repeat_interleave(G, dim=1)
+        vr = vt.repeat_interleave(G, dim=1)
+        ms = attempt(kr, vr, False)
+        del kr, vr
+        return {"ms": ms, "kernel": "torch sdpa (kv heads repeated)", "enable_gqa_error": first}
+    except RuntimeError as exc:
+        return {"error": str(exc).splitlines()[0][:200]}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -282,18 +401,33 @@ def run_moba(args):
     if dist:
         dist.barrier()
     import block_sparse_long_gate_b200 as moba
+    from block_sparse_long_gate_b200 import flops as fx
+    from block_sparse_long_gate_b200 import partition
 
     moba.lib()
-    w = workload(args.seq_len, args.hq, args.hkv)
+    w = workload(args.seq_len, args.hq, args.hkv, args.config)
     B, N, Hq, Hkv, d, bs, topk = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], w["block_size"], w["topk"]
-    seed = w["seed"] + rank
-
-    q_h, k_h, v_h = host_inputs(w, seed, pin=True)
+    split = world > 1 and partition.can_split(Hq, Hkv, world)
+    if split:  # one forward, split by kv-head groups
+        sl = partition.head_slices(Hq, Hkv, world)[rank]
+        hq_r, hkv_r, seed = sl.n_q, sl.n_kv, w["seed"]
+        q_h, k_h, v_h = host_inputs(w, seed, pin=True, hkv_range=(sl.hkv0, sl.hkv1))
+        parallelism = (f"one forward split over {world} GPUs by kv-head groups (rank {rank}: kv heads "
+                       f"[{sl.hkv0}, {sl.hkv1}) and their query heads), no collective on the data path")
+        scaling = "strong"
+    else:  # independent forwards (world 1, or fewer kv heads than ranks)
+        hq_r, hkv_r, seed = Hq, Hkv, w["seed"] + rank
+        q_h, k_h, v_h = host_inputs(w, seed, pin=True)
+        parallelism = ("single GPU" if world == 1 else
+                       f"{world} independent forwards, one per GPU (seed + rank), no collective")
+        scaling = "weak"
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     out = torch.empty_like(q)
-    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
-    ws = torch.empty(moba.workspace_size(B, Hq, Hkv, N, d, bs, topk), dtype=torch.uint8, device=dev)
+    lse = torch.empty((B, hq_r, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(moba.workspace_size(B, hq_r, hkv_r, N, d, bs, topk), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    in_bytes = (q.numel() + k.numel() + v.numel()) * 2
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if in_bytes < L2_FLUSH_BELOW else None
 
     def step():
         moba.forward(q, k, v, bs, topk, out=out, lse=lse, workspace=ws)
@@ -308,16 +442,22 @@ def run_moba(args):
     gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local_rank)
     moba.stage_timing(True)
     launches0 = moba.launch_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     with ClockSampler(gpu_id) as clk:
         if dist:
             dist.barrier()
         torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
+        if flush is None:
+            ev[0][0].record(stream)
+            for _ in range(args.steps):
+                step()
+            ev[0][1].record(stream)
+        else:  # small inputs: rewrite a 256 MB buffer (twice the L2) between timed steps
+            for a, b in ev:
+                flush.fill_(1)
+                a.record(stream)
+                step()
+                b.record(stream)
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
@@ -325,9 +465,9 @@ def run_moba(args):
     stages, calls = moba.stage_times()
     moba.stage_timing(False)
     status = moba.sync_status()
-    local_ms = e0.elapsed_time(e1)
-    fl = useful_flops(w)
-    total_ms, total_flops = aggregate(local_ms, fl * args.steps, world)
+    local_ms = ev[0][0].elapsed_time(ev[0][1]) if flush is None else sum(a.elapsed_time(b) for a, b in ev)
+    fl_local = fx.useful_flops(B, hq_r, N, d, bs, topk)
+    total_ms, total_flops = aggregate(local_ms, fl_local * args.steps, world)
     value = total_flops / (total_ms * 1e-3) / 1e12
     ms_per_step = total_ms / args.steps
 
@@ -343,7 +483,7 @@ def run_moba(args):
         out_h.copy_(out, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
 
-    h2d = (q.numel() + k.numel() + v.numel()) * 2
+    h2d = in_bytes
     d2h = out.numel() * 2 + lse.numel() * 4
     e2e = None
     if args.e2e_steps > 0:
@@ -351,39 +491,54 @@ def run_moba(args):
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
+        e0, e1 = ev[0]
         e0.record(stream)
         for _ in range(args.e2e_steps):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms, e2e_flops = aggregate(e0.elapsed_time(e1), fl * args.e2e_steps, world)
+        e2e_ms, e2e_flops = aggregate(e0.elapsed_time(e1), fl_local * args.e2e_steps, world)
         e2e = {"value": e2e_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps, "ms_per_step": e2e_ms / args.e2e_steps}
 
-    # dense causal attention of the same shape on the same GPU (our tcgen05 kernel), once
+    # dense causal attention of the same shape on the same GPU: this library's tcgen05 kernel and
+    # torch's fused attention, each once (the whole shape, on rank 0 only)
     dense = None
-    if not args.no_dense and rank == 0:
+    if not args.no_dense and rank == 0 and not split:
         del ws
         torch.cuda.empty_cache()
         dout, dlse = torch.empty_like(q), torch.empty_like(lse)
         moba.dense_causal(q[:, :4096].contiguous(), k[:, :4096].contiguous(), v[:, :4096].contiguous())
         torch.cuda.synchronize()
+        e0, e1 = ev[0]
+        if flush is not None:
+            flush.fill_(1)
         e0.record(stream)
         moba.dense_causal(q, k, v, out=dout, lse=dlse)
         e1.record(stream)
         torch.cuda.synchronize()
-        from block_sparse_long_gate_b200 import flops as fx
         dms = e0.elapsed_time(e1)
-        dense = {"ms": dms, "tflops": fx.dense_causal_flops(B, Hq, N, d) / dms / 1e9, "kernel": "moba_dense_causal"}
-        del dout, dlse
+        dflops = fx.dense_causal_flops(B, Hq, N, d)
+        dense = {"moba_dense_causal": {"ms": dms, "tflops": dflops / dms / 1e9}}
         if moba.sync_status() != 0:
-            dense["status"] = "device error"
+            dense["moba_dense_causal"]["status"] = "device error"
+        del dout, dlse
+        torch.cuda.empty_cache()
+        if not args.no_sdpa:
+            sd = time_sdpa(q, k, v, stream)
+            if "ms" in sd:
+                sd["tflops"] = dflops / sd["ms"] / 1e9
+            dense["torch_sdpa"] = sd
+        best = min((x for x in dense.values() if "ms" in x), key=lambda x: x["ms"])
+        dense["fastest"] = [n for n, x in dense.items() if x is best][0]
+        dense["ms"] = best["ms"]
 
     peaks, peak_src = read_peaks()
-    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     attn_ms = stages["attention"] / max(calls, 1)
-    achieved = fl / (attn_ms * 1e-3) / 1e12
-    traffic = attention_traffic()
+    achieved = fl_local / (attn_ms * 1e-3) / 1e12
+    traffic = attention_traffic() if (w["config"] == DEFAULT_CONFIG and N == WORKLOAD["N"]
+                                      and Hq == WORKLOAD["Hq"] and not split) else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -391,30 +546,31 @@ def run_moba(args):
         torch.cuda.empty_cache()
         secs, sfl, nrows = oracle_sample(q_h, k_h, v_h, w, args.sample_rows, 77)
         cpu = {"value": sfl / secs / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-               "sample": f"{nrows} seeded rows over all heads and the whole sequence (pool of all of K, then "
-                         f"gate + attend of the sampled rows, fp64), {secs:.1f} s"}
+               "sample": sample_text(w, nrows) + f", {secs:.1f} s"}
 
     if rank == 0:
         clocks = clk.summary()
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "metric": metric_name(w), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": scaling,
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": workload_name(w),
-                       "global_batch": B * world, "seq_len": N,
-                       "parallelism": f"{world} independent forward(s), one per GPU, no collective",
-                       "l2": "inputs (12 GiB) far exceed the 126 MB L2; no flush between steps"},
-            "pct_of_peak": 100.0 * value / world / peak,
-            "peak_tflops": peak, "peak_source": f"bf16_tflops_sustained of {peak_src}",
+                       "global_batch": B * (1 if split else world), "seq_len": N, "parallelism": parallelism,
+                       "l2": ("inputs far exceed the 126 MB L2; no flush between steps" if flush is None else
+                              "a 256 MB buffer is rewritten before every timed step (L2 flush), "
+                              "steps timed one by one")},
+        }
+        line.update(peak_fields(value / world, clocks, peaks, peak_src))
+        line.update({
             "stages_ms_per_step": {s: t / max(calls, 1) for s, t in stages.items()},
-            "roofline": {"kernel": "moba_attn_tc_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"bf16_tflops_sustained, {peak_src}"},
+            "roofline": {"kernel": "moba_attn_tc_kernel", "bound": "tensor", "achieved": achieved, "peak": sust,
+                         "unit": "TFLOP/s", "frac": achieved / sust, "traffic": traffic,
+                         "peak_source": f"bf16_tflops_sustained (kernel timed inside a long step), {peak_src}"},
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clocks,
             "device_status": status,
-        }
+        })
         if dense:
             line["dense"] = dense
             line["speedup_vs_dense"] = dense["ms"] / ms_per_step

@@ -53,6 +53,11 @@ def _load():
             lib.synth_key_offset.argtypes = [ctypes.c_uint64] + [ctypes.c_int64] * 5
             lib.synth_fill_keys.restype = None
             lib.synth_fill_keys.argtypes = [ctypes.c_void_p, ctypes.c_uint64] + [ctypes.c_int64] * 5
+            lib.synth_fill_normal_heads.restype = None
+            lib.synth_fill_normal_heads.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint32] + \
+                [ctypes.c_int64] * 6
+            lib.synth_fill_keys_heads.restype = None
+            lib.synth_fill_keys_heads.argtypes = [ctypes.c_void_p, ctypes.c_uint64] + [ctypes.c_int64] * 7
             _lib = lib
     return _lib
 
@@ -84,6 +89,22 @@ def inputs(B: int, N: int, Hq: int, Hkv: int, d: int, block_size: int, seed: int
     q = normal(seed, Q_ID, (B, N, Hq, d), pin)
     k = keys(seed, B, N, Hkv, d, block_size, pin)
     v = normal(seed, V_ID, (B, N, Hkv, d), pin)
+    return q, k, v
+
+
+def inputs_heads(B: int, N: int, Hq: int, Hkv: int, d: int, block_size: int, seed: int, hkv0: int, hkv1: int,
+                 pin: bool = False):
+    """The slice of `inputs(...)` a rank owning kv heads [hkv0, hkv1) needs: q of query heads
+    [hkv0 * G, hkv1 * G) (G = Hq / Hkv) and k, v of kv heads [hkv0, hkv1), each contiguous and
+    equal element for element to that slice of the whole tensors."""
+    G = Hq // Hkv
+    L = _load()
+    q = _empty((B, N, (hkv1 - hkv0) * G, d), pin)
+    L.synth_fill_normal_heads(q.data_ptr(), seed, Q_ID, B, N, Hq, d, hkv0 * G, hkv1 * G)
+    k = _empty((B, N, hkv1 - hkv0, d), pin)
+    L.synth_fill_keys_heads(k.data_ptr(), seed, B, N, Hkv, d, block_size, hkv0, hkv1)
+    v = _empty((B, N, hkv1 - hkv0, d), pin)
+    L.synth_fill_normal_heads(v.data_ptr(), seed, V_ID, B, N, Hkv, d, hkv0, hkv1)
     return q, k, v
 
 

@@ -108,3 +108,37 @@ void synth_fill_keys(uint16_t* out, uint64_t seed, int64_t B, int64_t N, int64_t
         }
     }
 }
+
+/* Heads [h0, h1) of the N(0,1) tensor [B, N, H, d] of stream (seed, tensor_id), written as
+ * [B, N, h1 - h0, d]: element (b, t, h, e) is number ((b * N + t) * H + h) * d + e of the
+ * stream, the same value the whole tensor holds there. */
+void synth_fill_normal_heads(uint16_t* out, uint64_t seed, uint32_t tensor_id, int64_t B, int64_t N,
+                             int64_t H, int64_t d, int64_t h0, int64_t h1) {
+    uint64_t key = synth_stream_key(seed, tensor_id);
+    int64_t nh = h1 - h0;
+#pragma omp parallel for schedule(static)
+    for (int64_t row = 0; row < B * N * nh; ++row) {
+        int64_t h = h0 + row % nh;
+        int64_t bt = row / nh;
+        for (int64_t e = 0; e < d; ++e)
+            out[row * d + e] = synth_bf16_rne(synth_normal_at(key, (uint64_t)((bt * H + h) * d + e)));
+    }
+}
+
+/* Heads [h0, h1) of the key tensor of synth_fill_keys, written as [B, N, h1 - h0, d]. */
+void synth_fill_keys_heads(uint16_t* out, uint64_t seed, int64_t B, int64_t N, int64_t Hkv, int64_t d,
+                           int64_t block_size, int64_t h0, int64_t h1) {
+    uint64_t key = synth_stream_key(seed, SYNTH_K);
+    int64_t nblk = (N + block_size - 1) / block_size;
+    int64_t nh = h1 - h0;
+#pragma omp parallel for schedule(static)
+    for (int64_t row = 0; row < B * N * nh; ++row) {
+        int64_t h = h0 + row % nh;
+        int64_t t = (row / nh) % N;
+        int64_t b = row / (nh * N);
+        double c = synth_key_offset(seed, b, h, t / block_size, Hkv, nblk);
+        int64_t grow = (b * N + t) * Hkv + h;
+        for (int64_t e = 0; e < d; ++e)
+            out[row * d + e] = synth_bf16_rne(synth_normal_at(key, (uint64_t)(grow * d + e)) + c);
+    }
+}
