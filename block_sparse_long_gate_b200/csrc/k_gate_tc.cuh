@@ -10,22 +10,29 @@
 // times the row sum in fp32 plus a tcgen05 contraction of the exact bf16 query
 // tile with the residual r_j = Kbar_j - mu_j held as two bf16 planes (hi, lo),
 // accumulated in fp32 in TMEM. |s~_j - s_j| <= eps, a bound derived from the
-// magnitudes involved (computed per row before the boundary pass). One thread owns one query row and keeps
-// the best k - 1 + GATE_EXTRA candidates by s~. Every candidate whose s~ lies
-// within 2 eps of the (k-1)-th best is re-scored exactly (fp64, the same
-// evaluation as the fp64 gate), which decides the boundary exactly:
-//   - candidates with s~ > T + 2 eps are certainly kept,
-//   - the exact top list needs nothing below T - 2 eps,
-// where T is the (k-1)-th best s~. If the kept list cannot show that nothing
-// below it reaches T - 2 eps, the row is re-scored exactly over all candidates.
+// magnitudes involved (computed per row before its scan). One thread owns one
+// query row and keeps the best k - 1 + GATE_EXTRA candidates in a sorted list of
+// 32-bit keys: the score on a per-row grid of 2^18 levels over the bound
+// [-R, R] of |s~| (top 18 bits) and 16383 - j (low 14 bits), so one unsigned
+// compare orders two candidates by (grid level desc, block index asc) and an
+// insertion is a chain of integer max / min pairs. sigma(key), the grid level's
+// value, is within eps' = eps + 2 h of the exact score (h = grid step). Every
+// candidate whose sigma lies within 2 eps' of the (k-1)-th best is re-scored
+// exactly (fp64, the same evaluation as the fp64 gate), which decides the
+// boundary exactly:
+//   - candidates with sigma > T + 2 eps' are certainly kept,
+//   - the exact top list needs nothing below T - 2 eps',
+// where T is sigma of the (k-1)-th best key. If the kept list cannot show that
+// nothing below it reaches T - 2 eps' (or a score fell off the grid), the row
+// is re-scored exactly over all candidates.
 //
 // Roles (192 threads, persistent over 128-token tiles of one query head):
 //   warp 0     TMA: Q tile (3-D map over [d, Hq, B*N]),
-//              residual planes of 64 candidate blocks per step into 2 stages
-//   warp 1     tcgen05.mma issuer: S (128 rows x 64 candidates, fp32) = sum over
+//              residual planes of 32 candidate blocks per step into 2 stages
+//   warp 1     tcgen05.mma issuer: S (128 rows x 32 candidates, fp32) = sum over
 //              the two planes and 8 K-steps of Q x plane^T, into 2 TMEM buffers
 //   warps 2-5  top-k: one thread per row (TMEM lane)
-// Shared memory (~113 KB) and TMEM (128 columns) are sized so that two CTAs
+// Shared memory (~74 KB) and TMEM (64 columns) are sized so that three CTAs
 // share an SM and hide each other's latencies.
 #pragma once
 #include <cuda.h>
@@ -34,17 +41,24 @@
 #include "k_pool.cuh"
 
 #define GATE_TC_THREADS 192
+#define GATE_TC_CTAS 3                    // CTAs per SM
 #define GATE_EXTRA 4
-#define GATE_CAND 64                      // candidate blocks per step (MMA N)
+#define GATE_CAND 32                      // candidate blocks per step (MMA N)
 #define GATE_Q_BYTES 32768
-#define GATE_STAGE_BYTES 32768            // 2 planes x 64 rows x 256 B
+#define GATE_PLANE_BYTES (GATE_CAND * 256)  // one bf16 plane of GATE_CAND rows x 128 features
+#define GATE_STAGE_BYTES (2 * GATE_PLANE_BYTES)
 #define GATE_GROUP 16                    // scores staged per TMEM load
 #define GATE_SV_BYTES (GATE_GROUP * 128 * 4)
-#define GATE_TC_SMEM (GATE_Q_BYTES + 2 * GATE_STAGE_BYTES + GATE_SV_BYTES + 1024 + 256)  // 2 CTAs per SM
+#define GATE_TC_SMEM (GATE_Q_BYTES + 2 * GATE_STAGE_BYTES + GATE_SV_BYTES + 1024 + 256)
+#define GATE_TMEM_COLS 64                 // 2 score buffers of GATE_CAND columns
+#define GATE_QBITS 18                     // score grid levels: 2^18
+#define GATE_JBITS 14                     // block index bits of a key (MOBA_MAX_BLOCKS = 2^14)
+static_assert(MOBA_MAX_BLOCKS <= (1 << GATE_JBITS), "block index does not fit the key");
+static_assert(GATE_QBITS + GATE_JBITS == 32, "keys are 32-bit");
 
 struct __align__(64) GateMaps {
     CUtensorMap q;       // (d, Hq, B*N), box (64, 1, 128)
-    CUtensorMap planes;  // (d, B*Hkv*2*nfull), box (64, 64)
+    CUtensorMap planes;  // (d, B*Hkv*2*nfull), box (64, GATE_CAND)
 };
 
 struct GateParams {
@@ -120,13 +134,13 @@ __device__ unsigned long long g_gate_stats[4];  // rows scored, zone re-scores, 
 #endif
 
 template <int KPX>
-__global__ void __launch_bounds__(GATE_TC_THREADS, 2)
+__global__ void __launch_bounds__(GATE_TC_THREADS, GATE_TC_CTAS)
     moba_gate_tc_kernel(const GateParams p, const __grid_constant__ GateMaps maps) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* sQ = smem;                     // 32 KB
-    uint8_t* sC = smem + GATE_Q_BYTES;      // 2 x 32 KB
-    float* sV = (float*)(smem + GATE_Q_BYTES + 2 * GATE_STAGE_BYTES);  // [GATE_GROUP][128] score staging
+    uint8_t* sC = smem + GATE_Q_BYTES;      // 2 stages of GATE_STAGE_BYTES
+    uint32_t* sV = (uint32_t*)(smem + GATE_Q_BYTES + 2 * GATE_STAGE_BYTES);  // [GATE_GROUP][128] key staging
     GateBars* bars = (GateBars*)(smem + GATE_Q_BYTES + 2 * GATE_STAGE_BYTES + GATE_SV_BYTES);
     volatile int* abort_flag = &bars->abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -147,7 +161,7 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, 2)
         fence_mbarrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(&bars->tmem_base, 128);
+        tmem_alloc(&bars->tmem_base, GATE_TMEM_COLS);
         tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
@@ -182,8 +196,9 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, 2)
 #pragma unroll
                     for (int pl = 0; pl < 2; ++pl) {
                         const int r = (int)((bh * 2 + pl) * p.nfull + (int64_t)m * GATE_CAND);
-                        tma_load_3d(smem_u32(st + pl * 16384), &maps.planes, &bars->c_full[s], 0, 0, r);
-                        tma_load_3d(smem_u32(st + pl * 16384 + 8192), &maps.planes, &bars->c_full[s], 64, 0, r);
+                        uint8_t* dst = st + pl * GATE_PLANE_BYTES;
+                        tma_load_3d(smem_u32(dst), &maps.planes, &bars->c_full[s], 0, 0, r);
+                        tma_load_3d(smem_u32(dst + GATE_PLANE_BYTES / 2), &maps.planes, &bars->c_full[s], 64, 0, r);
                     }
                     bars->issued_c[s] += 1;
                 }
@@ -217,7 +232,8 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, 2)
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const uint32_t qoff = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
-                        const uint32_t coff = (pl * 16384 + (k >> 2) * 8192 + (k & 3) * 32) >> 4;
+                        const uint32_t coff =
+                            (pl * GATE_PLANE_BYTES + (k >> 2) * (GATE_PLANE_BYTES / 2) + (k & 3) * 32) >> 4;
                         tc_mma_ss_w(tS, dq + qoff, dc + coff, idesc, (pl > 0 || k > 0) ? 1u : 0u);
                     }
                 tc_commit_w(&bars->c_empty[s]);
@@ -243,7 +259,6 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, 2)
             const int64_t t = gt.t0 + r;
             const int64_t c = active ? t / p.bs : 0;
             const bool need = active && kp > 0 && c > kp;
-            const int64_t bh = (int64_t)gt.b * p.Hkv + gt.hk;
             const uint8_t* qrow = sQ + r * 128;  // this row of the swizzled tile
             // row sum and l1 norm (exact in fp64)
             double sq64 = 0.0, l1 = 0.0;
@@ -259,16 +274,23 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, 2)
                 }
             }
             const float sq = (float)sq64;
-            float ts[KPX];
-            int tj[KPX];
+            // Bounds of this row (see the file comment): |s| <= Rd, |s~ - s| <= eps <= Rd, so
+            // |s~| <= Rb = Rd + eps; the key grid spans [-Rb, Rb] with step h.
+            const int64_t bh = (int64_t)gt.b * p.Hkv + gt.hk;
+            const double mu_max = (double)__uint_as_float(p.stats[bh * 2 + 0]);
+            const double r_max = (double)__uint_as_float(p.stats[bh * 2 + 1]);
+            const double Rd = mu_max * fabs(sq64) + l1 * r_max;
+            const double eps = 0x1p-11 * l1 * r_max + 0x1p-20 * (mu_max * fabs(sq64) + 2.0 * Rd) + 1e-30;
+            const double Rb = Rd + eps;
+            const uint32_t qmax = (1u << GATE_QBITS) - 1u;
+            // x = s~ * inv_h + off lands in [1, qmax]; level q = floor(x)
+            const float inv_h = (float)((double)(qmax - 2u) / (2.0 * Rb));
+            const float off = (float)(Rb * (double)inv_h + 1.0);
+            uint32_t ts[KPX];
 #pragma unroll
-            for (int i = 0; i < KPX; ++i) {
-                ts[i] = -INFINITY;
-                tj[i] = 0x7FFFFFFF;
-            }
-            float thr = -INFINITY;
-            int filled = 0;
-            float smax = 0.f;
+            for (int i = 0; i < KPX; ++i) ts[i] = 0u;  // 0: empty (every real key is >= 2^14)
+            uint32_t thr = 0u;
+            bool off_grid = false;
             const float* mu = p.mu + bh * p.nfull;
             bool ok = true;
             for (int m = 0; m < gt.nch; ++m, ++g) {
@@ -277,43 +299,40 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, 2)
                 tc_fence_after();
                 const int64_t j0 = (int64_t)m * GATE_CAND;
                 const int jend = need ? (int)((c - j0 < GATE_CAND) ? c - j0 : GATE_CAND) : 0;  // candidates j < c
-                float* sv = sV + r;  // this row's staged scores, stride 128 (bank = row)
+                const uint32_t kbase = (uint32_t)((1 << GATE_JBITS) - 1) - (uint32_t)j0;  // 16383 - j0
+                uint32_t* sv = sV + r;  // this row's staged keys, stride 128 (bank = row)
 #pragma unroll 1
                 for (int cc = 0; cc < GATE_CAND / GATE_GROUP; ++cc) {
                     uint32_t sr[GATE_GROUP];
                     tmem_ld16(tmem + s * GATE_CAND + lane_off + cc * GATE_GROUP, sr);
                     tc_wait_ld();
-                    // unrolled pass: scores and the candidates that beat the current threshold
+                    // unrolled pass: keys, and the candidates that beat the list's last key
                     uint32_t hits = 0;
 #pragma unroll
                     for (int jj = 0; jj < GATE_GROUP; ++jj) {
                         const int col = cc * GATE_GROUP + jj;
                         if (col < jend) {
                             const float v = fmaf(__ldg(mu + j0 + col), sq, __uint_as_float(sr[jj]));
-                            smax = fmaxf(smax, fabsf(v));
-                            sv[jj * 128] = v;
-                            if (v > thr) hits |= 1u << jj;
+                            const uint32_t lvl = __float2uint_rz(fmaf(v, inv_h, off));
+                            off_grid |= (lvl - 1u) > (qmax - 1u);  // outside [1, qmax]
+                            const uint32_t key = (lvl << GATE_JBITS) + (kbase - (uint32_t)col);
+                            sv[jj * 128] = key;
+                            if (key > thr) hits |= 1u << jj;
                         }
                     }
                     // one insertion chain in the code, entered once per hit in ascending block order
                     while (hits) {
                         const int jj = __ffs(hits) - 1;
                         hits &= hits - 1;
-                        float cs = sv[jj * 128];
-                        if (!(cs > thr)) continue;
-                        int cj = (int)(j0 + cc * GATE_GROUP + jj);
+                        uint32_t x = sv[jj * 128];
+                        if (x <= thr) continue;
 #pragma unroll
                         for (int i = 0; i < KPX; ++i) {
-                            if (cs > ts[i] || (cs == ts[i] && cj < tj[i])) {
-                                const float x = ts[i];
-                                ts[i] = cs;
-                                cs = x;
-                                const int y = tj[i];
-                                tj[i] = cj;
-                                cj = y;
-                            }
+                            const uint32_t hi = max(ts[i], x);
+                            x = min(ts[i], x);
+                            ts[i] = hi;
                         }
-                        if (++filled >= KPX) thr = ts[KPX - 1];
+                        thr = ts[KPX - 1];
                     }
                 }
                 tc_fence_before();
@@ -329,33 +348,36 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, 2)
                         orow[0] = (int32_t)c;
                     }
                 } else {
-                    // error bound of s~ (see the file comment): tensor-core accumulation of the residual
-                    // part and its two-plane representation, plus the fp32 centre product and sum.
-                    const float mu_max = __uint_as_float(p.stats[bh * 2 + 0]);
-                    const float r_max = __uint_as_float(p.stats[bh * 2 + 1]);
-                    const double eps = 0x1p-11 * l1 * (double)r_max +
-                                       0x1p-20 * ((double)mu_max * fabs(sq64) + (double)smax) + 1e-30;
-                    float T = 0.f;
+                    // grid value of a key and its distance bound eps' to the exact score
+                    const double hd = 1.0 / (double)inv_h, offd = (double)off;
+                    auto sigma = [&](uint32_t key) { return ((double)(key >> GATE_JBITS) - offd) * hd; };
+                    auto block_of = [&](uint32_t key) {
+                        return (int)(((1u << GATE_JBITS) - 1u) - (key & ((1u << GATE_JBITS) - 1u)));
+                    };
+                    const double epsq = eps + 2.0 * hd;
+                    uint32_t Tk = 0u;
 #pragma unroll
                     for (int i = 0; i < KPX; ++i)
-                        if (i == kp - 1) T = ts[i];
-                    const double lo_thr = (double)T - 2.0 * eps, hi_thr = (double)T + 2.0 * eps;
+                        if (i == kp - 1) Tk = ts[i];
+                    const double T = sigma(Tk);
+                    const double lo_thr = T - 2.0 * epsq, hi_thr = T + 2.0 * epsq;
                     const double* kb = p.kbar + bh * p.nfull * MOBA_D;
-                    const bool overflow = (c > KPX) && ((double)ts[KPX - 1] >= lo_thr);
+                    const bool overflow = off_grid || ((c > KPX) && sigma(ts[KPX - 1]) >= lo_thr);
                     GATE_STAT(0, 1);
                     GATE_STAT(2, overflow ? 1 : 0);
                     // kept blocks (local array, filled in any order, sorted at the end)
                     int outj[KPX];
                     int nout = 0;
-                    // exact candidates: the band [T - 2 eps, T + 2 eps], or every candidate on overflow
+                    // exact candidates: the band [T - 2 eps', T + 2 eps'], or every candidate on overflow
                     int bj[KPX];
                     int nb = 0;
                     if (!overflow) {
 #pragma unroll
                         for (int i = 0; i < KPX; ++i) {
-                            const bool valid = tj[i] != 0x7FFFFFFF;
-                            if (valid && (double)ts[i] > hi_thr) outj[nout++] = tj[i];  // certainly kept
-                            else if (valid && (double)ts[i] >= lo_thr) bj[nb++] = tj[i];
+                            const bool valid = ts[i] != 0u;
+                            const double si = sigma(ts[i]);
+                            if (valid && si > hi_thr) outj[nout++] = block_of(ts[i]);  // certainly kept
+                            else if (valid && si >= lo_thr) bj[nb++] = block_of(ts[i]);
                         }
                     }
                     const int need_n = kp - nout;
@@ -409,7 +431,7 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, 2)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 128);
+    if (warp == 1) tmem_dealloc(tmem, GATE_TMEM_COLS);
 }
 
 // ---------------------------------------------------------------- host side
@@ -449,7 +471,7 @@ static int run_gate_tc(const GateParams& gp, const uint16_t* planes, cudaStream_
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return MOBA_ERR_CUDA;
-    const int grid = (int)(gp.ntiles < 2 * nsm ? gp.ntiles : 2 * nsm);
+    const int grid = (int)(gp.ntiles < GATE_TC_CTAS * nsm ? gp.ntiles : GATE_TC_CTAS * nsm);
     if (gp.kp + GATE_EXTRA <= 8) return launch_gate_tc<8>(gp, maps, grid, st);
     if (gp.kp + GATE_EXTRA <= 16) return launch_gate_tc<16>(gp, maps, grid, st);
     if (gp.kp + GATE_EXTRA <= 24) return launch_gate_tc<24>(gp, maps, grid, st);
