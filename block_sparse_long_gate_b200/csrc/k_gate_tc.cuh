@@ -48,8 +48,12 @@
 #define GATE_PLANE_BYTES (GATE_CAND * 256)  // one bf16 plane of GATE_CAND rows x 128 features
 #define GATE_STAGE_BYTES (2 * GATE_PLANE_BYTES)
 #define GATE_GROUP 16                    // scores staged per TMEM load
-#define GATE_SV_BYTES (GATE_GROUP * 128 * 4)
-#define GATE_TC_SMEM (GATE_Q_BYTES + 2 * GATE_STAGE_BYTES + GATE_SV_BYTES + 1024 + 256)
+// Per-row staging column in shared memory (stride 128 words, so row r's words sit in bank r):
+// the keys of one TMEM load during the scan, then the boundary band and the sorted output.
+__host__ __device__ constexpr int gate_sv_rows(int kpx) { return kpx > GATE_GROUP ? kpx : GATE_GROUP; }
+__host__ __device__ constexpr int gate_tc_smem(int kpx) {
+    return GATE_Q_BYTES + 2 * GATE_STAGE_BYTES + gate_sv_rows(kpx) * 128 * 4 + 1024 + 256;
+}
 #define GATE_TMEM_COLS 64                 // 2 score buffers of GATE_CAND columns
 #define GATE_QBITS 18                     // score grid levels: 2^18
 #define GATE_JBITS 14                     // block index bits of a key (MOBA_MAX_BLOCKS = 2^14)
@@ -102,30 +106,6 @@ __device__ __forceinline__ GateTile gate_tile(const GateParams& p, int64_t item)
     return g;
 }
 
-// Exact fp64 score of one candidate for the thread's query row, reading the row from
-// the swizzled Q tile in shared memory (same evaluation order as the fp64 gate:
-// features ascending, one fused multiply-add each).
-__device__ __forceinline__ double exact_score(const uint8_t* qrow, int r, const double* kb) {
-    double s = 0.0;
-#pragma unroll 2
-    for (int ch = 0; ch < 16; ++ch) {
-        const uint4 v = *reinterpret_cast<const uint4*>(qrow + (ch >> 3) * 16384 + (((ch & 7) ^ (r & 7)) << 4));
-        const double2 k0 = __ldg(reinterpret_cast<const double2*>(kb + ch * 8));
-        const double2 k1 = __ldg(reinterpret_cast<const double2*>(kb + ch * 8 + 2));
-        const double2 k2 = __ldg(reinterpret_cast<const double2*>(kb + ch * 8 + 4));
-        const double2 k3 = __ldg(reinterpret_cast<const double2*>(kb + ch * 8 + 6));
-        s = fma((double)bf16lo(v.x), k0.x, s);
-        s = fma((double)bf16hi(v.x), k0.y, s);
-        s = fma((double)bf16lo(v.y), k1.x, s);
-        s = fma((double)bf16hi(v.y), k1.y, s);
-        s = fma((double)bf16lo(v.z), k2.x, s);
-        s = fma((double)bf16hi(v.z), k2.y, s);
-        s = fma((double)bf16lo(v.w), k3.x, s);
-        s = fma((double)bf16hi(v.w), k3.y, s);
-    }
-    return s;
-}
-
 #ifdef MOBA_GATE_STATS
 __device__ unsigned long long g_gate_stats[4];  // rows scored, zone re-scores, full re-scores, zone size sum
 #define GATE_STAT(i, v) atomicAdd(&g_gate_stats[i], (unsigned long long)(v))
@@ -140,8 +120,8 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, GATE_TC_CTAS)
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* sQ = smem;                     // 32 KB
     uint8_t* sC = smem + GATE_Q_BYTES;      // 2 stages of GATE_STAGE_BYTES
-    uint32_t* sV = (uint32_t*)(smem + GATE_Q_BYTES + 2 * GATE_STAGE_BYTES);  // [GATE_GROUP][128] key staging
-    GateBars* bars = (GateBars*)(smem + GATE_Q_BYTES + 2 * GATE_STAGE_BYTES + GATE_SV_BYTES);
+    uint32_t* sV = (uint32_t*)(smem + GATE_Q_BYTES + 2 * GATE_STAGE_BYTES);  // [gate_sv_rows][128] staging
+    GateBars* bars = (GateBars*)(smem + GATE_Q_BYTES + 2 * GATE_STAGE_BYTES + gate_sv_rows(KPX) * 128 * 4);
     volatile int* abort_flag = &bars->abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -339,6 +319,8 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, GATE_TC_CTAS)
                 mbar_arrive(&bars->s_empty[s]);
             }
             if (!ok) break;
+            bool overflow = false, slow = false;
+            int ncert = 0, nband = 0, need_n = 0;
             if (active) {
                 int32_t* orow = p.idx + (((int64_t)gt.b * p.Hq + gt.hq) * p.N + t) * p.topk;
                 if (!need) {
@@ -361,62 +343,102 @@ __global__ void __launch_bounds__(GATE_TC_THREADS, GATE_TC_CTAS)
                         if (i == kp - 1) Tk = ts[i];
                     const double T = sigma(Tk);
                     const double lo_thr = T - 2.0 * epsq, hi_thr = T + 2.0 * epsq;
-                    const double* kb = p.kbar + bh * p.nfull * MOBA_D;
-                    const bool overflow = off_grid || ((c > KPX) && sigma(ts[KPX - 1]) >= lo_thr);
+                    overflow = off_grid || ((c > KPX) && sigma(ts[KPX - 1]) >= lo_thr);
                     GATE_STAT(0, 1);
                     GATE_STAT(2, overflow ? 1 : 0);
-                    // kept blocks (local array, filled in any order, sorted at the end)
-                    int outj[KPX];
-                    int nout = 0;
-                    // exact candidates: the band [T - 2 eps', T + 2 eps'], or every candidate on overflow
-                    int bj[KPX];
-                    int nb = 0;
-                    if (!overflow) {
+                    // the list is sorted by key, so the certainly kept entries come first, then the band
 #pragma unroll
-                        for (int i = 0; i < KPX; ++i) {
-                            const bool valid = ts[i] != 0u;
-                            const double si = sigma(ts[i]);
-                            if (valid && si > hi_thr) outj[nout++] = block_of(ts[i]);  // certainly kept
-                            else if (valid && si >= lo_thr) bj[nb++] = block_of(ts[i]);
-                        }
+                    for (int i = 0; i < KPX; ++i) {
+                        const double si = sigma(ts[i]);
+                        ncert += (ts[i] != 0u && si > hi_thr) ? 1 : 0;
+                        nband += (ts[i] != 0u && si >= lo_thr && si <= hi_thr) ? 1 : 0;
                     }
-                    const int need_n = kp - nout;
-                    // exact top need_n by (score desc, block index asc), insertion into a short list
-                    double es[KPX];
-                    int ej[KPX];
-                    int ne = 0;
-                    const int64_t n_exact = overflow ? c : nb;
-#pragma unroll 1
-                    for (int64_t z = 0; z < n_exact; ++z) {
-                        const int jz = overflow ? (int)z : bj[z];
-                        const double e = exact_score(qrow, r, kb + (int64_t)jz * MOBA_D);
-                        GATE_STAT(3, 1);
-                        int pos = ne;
-                        while (pos > 0 && (e > es[pos - 1] || (e == es[pos - 1] && jz < ej[pos - 1]))) --pos;
-                        if (pos >= need_n) continue;
-                        const int last = ne < need_n ? ne : need_n - 1;
-                        for (int u = last; u > pos; --u) {
-                            es[u] = es[u - 1];
-                            ej[u] = ej[u - 1];
-                        }
-                        es[pos] = e;
-                        ej[pos] = jz;
-                        if (ne < need_n) ++ne;
+                    if (overflow) ncert = 0;
+                    need_n = kp - ncert;
+                    // every band entry is kept when the band holds exactly the open slots (the
+                    // common case): then no exact score is needed
+                    slow = overflow || nband > need_n;
+                    if (slow && !overflow) {  // stage the band's blocks for the exact pass
+#pragma unroll
+                        for (int i = 0; i < KPX; ++i)
+                            if (i >= ncert && i < ncert + nband) sV[(i - ncert) * 128 + r] = (uint32_t)block_of(ts[i]);
                     }
-                    for (int u = 0; u < ne; ++u) outj[nout++] = ej[u];
-                    // ascending block order
-                    for (int i2 = 1; i2 < nout; ++i2) {
-                        const int v = outj[i2];
-                        int u = i2;
-                        while (u > 0 && outj[u - 1] > v) {
-                            outj[u] = outj[u - 1];
-                            --u;
-                        }
-                        outj[u] = v;
-                    }
-                    for (int i2 = 0; i2 < kp; ++i2) orow[i2] = outj[i2];
-                    orow[kp] = (int32_t)c;
                 }
+            }
+            // Exact fp64 scores of the rows that need them, one warp per score: lane e
+            // contracts features 4e..4e+3 and the warp sums the partials (a fixed order, so
+            // equal blocks score equally). The row that owns the candidates keeps the best
+            // need_n by (exact score desc, block index asc).
+            double es[KPX];
+            int ej[KPX];
+            int ne = 0;
+            {
+                const double* kbh = p.kbar + ((int64_t)gt.b * p.Hkv + gt.hk) * p.nfull * MOBA_D;
+                __syncwarp();  // the staged bands are visible to the whole warp
+                unsigned pend = __ballot_sync(0xffffffffu, slow);
+                while (pend) {
+                    const int L = __ffs(pend) - 1;
+                    pend &= pend - 1;
+                    const int rL = 32 * (warp & 3) + L;
+                    const bool ovL = __shfl_sync(0xffffffffu, overflow, L);
+                    const int nL = ovL ? (int)__shfl_sync(0xffffffffu, (int)c, L) : __shfl_sync(0xffffffffu, nband, L);
+                    const int needL = __shfl_sync(0xffffffffu, need_n, L);
+                    // this lane's four features of row rL (swizzled tile: 16-byte chunk lane / 2)
+                    const uint2 qv = *reinterpret_cast<const uint2*>(
+                        sQ + rL * 128 + ((lane >> 1) >> 3) * 16384 + ((((lane >> 1) & 7) ^ (rL & 7)) << 4) + (lane & 1) * 8);
+                    const double q0 = (double)bf16lo(qv.x), q1 = (double)bf16hi(qv.x);
+                    const double q2 = (double)bf16lo(qv.y), q3 = (double)bf16hi(qv.y);
+#pragma unroll 1
+                    for (int u = 0; u < nL; ++u) {
+                        const int jz = ovL ? u : (int)sV[u * 128 + rL];
+                        const double* kr = kbh + (int64_t)jz * MOBA_D + 4 * lane;
+                        const double2 a = __ldg(reinterpret_cast<const double2*>(kr));
+                        const double2 b2 = __ldg(reinterpret_cast<const double2*>(kr + 2));
+                        double e = q0 * a.x;
+                        e = fma(q1, a.y, e);
+                        e = fma(q2, b2.x, e);
+                        e = fma(q3, b2.y, e);
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+                        GATE_STAT(3, lane == 0 ? 1 : 0);
+                        if (lane == L) {
+                            int pos = ne;
+                            while (pos > 0 && (e > es[pos - 1] || (e == es[pos - 1] && jz < ej[pos - 1]))) --pos;
+                            if (pos < needL) {
+                                const int last = ne < needL ? ne : needL - 1;
+                                for (int z = last; z > pos; --z) {
+                                    es[z] = es[z - 1];
+                                    ej[z] = ej[z - 1];
+                                }
+                                es[pos] = e;
+                                ej[pos] = jz;
+                                if (ne < needL) ++ne;
+                            }
+                        }
+                    }
+                }
+                __syncwarp();  // every lane has read the staged bands before they are overwritten
+            }
+            if (need) {
+                // kept blocks in ascending order: insertion sort in this row's staging column
+                int32_t* orow = p.idx + (((int64_t)gt.b * p.Hq + gt.hq) * p.N + t) * p.topk;
+                uint32_t* srow = sV + r;
+                int n = 0;
+                auto put = [&](uint32_t v) {
+                    int u = n++;
+                    while (u > 0 && srow[(u - 1) * 128] > v) {
+                        srow[u * 128] = srow[(u - 1) * 128];
+                        --u;
+                    }
+                    srow[u * 128] = v;
+                };
+                const int nfirst = slow ? ncert : kp;  // leading list entries that are kept
+#pragma unroll
+                for (int i = 0; i < KPX; ++i)
+                    if (i < nfirst) put((uint32_t)(((1u << GATE_JBITS) - 1u) - (ts[i] & ((1u << GATE_JBITS) - 1u))));
+                for (int u = 0; u < ne; ++u) put((uint32_t)ej[u]);
+                for (int i2 = 0; i2 < kp; ++i2) orow[i2] = (int32_t)srow[i2 * 128];
+                orow[kp] = (int32_t)c;
             }
             mbar_arrive(&bars->q_empty);  // this row of the Q tile is no longer read
         }
@@ -450,9 +472,9 @@ static bool moba_make_2d_map(CUtensorMap* m, const void* base, int64_t rows) {
 template <int KPX>
 static int launch_gate_tc(const GateParams& gp, const GateMaps& maps, int grid, cudaStream_t st) {
     if (cudaFuncSetAttribute(moba_gate_tc_kernel<KPX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GATE_TC_SMEM) != cudaSuccess)
+                             gate_tc_smem(KPX)) != cudaSuccess)
         return MOBA_ERR_CUDA;
-    moba_gate_tc_kernel<KPX><<<grid, GATE_TC_THREADS, GATE_TC_SMEM, st>>>(gp, maps);
+    moba_gate_tc_kernel<KPX><<<grid, GATE_TC_THREADS, gate_tc_smem(KPX), st>>>(gp, maps);
     const cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) {
         cudaGetLastError();
