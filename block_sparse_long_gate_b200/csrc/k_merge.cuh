@@ -9,14 +9,15 @@
 //
 // HBM bound: per row (slots + 1) * (2d + 4) bytes read, 2d + 4 written. A
 // half-warp owns one row (16 lanes x 8 features, 16-byte accesses) and issues
-// the loads of up to 8 slots before it uses any of them, so enough bytes are in
-// flight to stream the partials at full bandwidth.
+// every load of the row (up to 16 slots) before it uses any of them, so a row
+// costs one memory latency and enough bytes are in flight to stream the
+// partials at full bandwidth.
 #pragma once
 #include "common.cuh"
 #include "k_invert.cuh"
 
 #define MERGE_THREADS 256
-#define MERGE_BATCH 8
+#define MERGE_BATCH 16
 
 __device__ __forceinline__ void fma8(float (&a)[8], float w, const uint4& x) {
     a[0] += w * bf16lo(x.x);
@@ -29,7 +30,13 @@ __device__ __forceinline__ void fma8(float (&a)[8], float w, const uint4& x) {
     a[7] += w * bf16hi(x.w);
 }
 
-// Merge of one row (b, hq, t) by one half-warp.
+// Merge of one row (b, hq, t) by one half-warp (lane i owns features 8i..8i+7).
+// Every load of the row is issued before any is used: the own partial, the slot
+// lse values and up to MERGE_BATCH slot partials, so a row costs one memory
+// latency. The slot count comes from the row's own block when the selection was
+// made by the library's gate (well formed by construction); an injected
+// selection (VALIDATE) is read and checked first.
+template <bool VALIDATE>
 __device__ __forceinline__ void merge_row(const int32_t* __restrict__ idx, const uint16_t* __restrict__ opart,
                                           const float* __restrict__ lpart, uint16_t* out, float* lse, int64_t N,
                                           int Hq, int bs, int topk, int64_t row) {
@@ -41,27 +48,37 @@ __device__ __forceinline__ void merge_row(const int32_t* __restrict__ idx, const
     const int64_t b = bh / Hq;
     const int kp = topk - 1;
     const int64_t c = t / bs;
-    const int32_t* sel = idx + row * topk;
-    const int p = check_row(sel, topk, c);
     uint16_t* orow = out + ((b * N + t) * Hq + hq) * MOBA_D + lane * 8;
-    if (p < 0) {
-        if (lane == 0) moba_set_error(MOBA_ERR_SELECTION);
-        *reinterpret_cast<uint4*>(orow) = make_uint4(0u, 0u, 0u, 0u);
-        if (lane == 0) lse[row] = __int_as_float(0x7fc00000);
-        return;
+    int p;
+    if (VALIDATE) {
+        p = check_row(idx + row * topk, topk, c);
+        if (p < 0) {
+            if (lane == 0) moba_set_error(MOBA_ERR_SELECTION);
+            *reinterpret_cast<uint4*>(orow) = make_uint4(0u, 0u, 0u, 0u);
+            if (lane == 0) lse[row] = __int_as_float(0x7fc00000);
+            return;
+        }
+    } else {
+        p = (int)(c < kp ? c : kp);
     }
     if (p == 0) return;  // only the own block: the partial already is the result
-    const float ld = lse[row];
     const float* lrow = lpart + row * kp;
-    // lane i holds lse of slots i, i + 16, i + 32, i + 48 (p <= 63)
+    const uint16_t* prow = opart + row * kp * MOBA_D + lane * 8;
+    // issue: own partial, slot lse values (lane i: slots i, i + 16, i + 32, i + 48), first batch
+    const uint4 dw = *reinterpret_cast<const uint4*>(orow);
+    const float ld = lse[row];
     float lsl[4];
-    float m = ld;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const int s = lane + 16 * r;
         lsl[r] = s < p ? lrow[s] : -INFINITY;
-        m = fmaxf(m, lsl[r]);
     }
+    uint4 x[MERGE_BATCH];
+#pragma unroll
+    for (int u = 0; u < MERGE_BATCH; ++u)
+        if (u < p) x[u] = *reinterpret_cast<const uint4*>(prow + (int64_t)u * MOBA_D);
+    // weights
+    float m = fmaxf(fmaxf(ld, lsl[0]), fmaxf(lsl[1], fmaxf(lsl[2], lsl[3])));
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(hmask, m, o));
     float z = 0.f;
@@ -77,26 +94,28 @@ __device__ __forceinline__ void merge_row(const int32_t* __restrict__ idx, const
     const float L = m + __logf(z);
     const float inv = 1.f / z;
     float acc[8];
-    {
-        const uint4 dw = *reinterpret_cast<const uint4*>(orow);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-        fma8(acc, wd, dw);
-    }
-    const uint16_t* prow = opart + row * kp * MOBA_D + lane * 8;
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    fma8(acc, wd, dw);
     const int src_base = (threadIdx.x & 16);
-    for (int s0 = 0; s0 < p; s0 += MERGE_BATCH) {
-        uint4 x[MERGE_BATCH];
+    auto weight = [&](int s) {
+        // weight of slot s lives in lane (s & 15), register s >> 4 of this half-warp
+        const float wr = (s >> 4) == 0 ? lsl[0] : (s >> 4) == 1 ? lsl[1] : (s >> 4) == 2 ? lsl[2] : lsl[3];
+        return __shfl_sync(hmask, wr, src_base + (s & 15));
+    };
+#pragma unroll
+    for (int u = 0; u < MERGE_BATCH; ++u) {
+        const float w = weight(u);
+        if (u < p) fma8(acc, w, x[u]);
+    }
+    for (int s0 = MERGE_BATCH; s0 < p; s0 += MERGE_BATCH) {  // long selections: further batches
 #pragma unroll
         for (int u = 0; u < MERGE_BATCH; ++u)
             if (s0 + u < p) x[u] = *reinterpret_cast<const uint4*>(prow + (int64_t)(s0 + u) * MOBA_D);
 #pragma unroll
         for (int u = 0; u < MERGE_BATCH; ++u) {
-            const int s = s0 + u;
-            // weight of slot s lives in lane (s & 15), register s >> 4 of this half-warp
-            const float wr = (s >> 4) == 0 ? lsl[0] : (s >> 4) == 1 ? lsl[1] : (s >> 4) == 2 ? lsl[2] : lsl[3];
-            const float w = __shfl_sync(hmask, wr, src_base + (s & 15));
-            if (s < p) fma8(acc, w, x[u]);
+            const float w = weight(s0 + u);
+            if (s0 + u < p) fma8(acc, w, x[u]);
         }
     }
     uint4 ow;
@@ -110,6 +129,7 @@ __device__ __forceinline__ void merge_row(const int32_t* __restrict__ idx, const
 
 // Persistent: each half-warp walks the rows with a stride of all half-warps of the grid
 // (short-lived blocks of a row each left the SMs partly idle between block launches).
+template <bool VALIDATE>
 __global__ void __launch_bounds__(MERGE_THREADS) moba_merge_kernel(const int32_t* __restrict__ idx,
                                                                    const uint16_t* __restrict__ opart,
                                                                    const float* __restrict__ lpart, uint16_t* out,
@@ -118,5 +138,5 @@ __global__ void __launch_bounds__(MERGE_THREADS) moba_merge_kernel(const int32_t
     const int64_t hw = (int64_t)blockIdx.x * (MERGE_THREADS / 16) + (threadIdx.x >> 4);
     const int64_t stride = (int64_t)gridDim.x * (MERGE_THREADS / 16);
     for (int64_t row = hw; row < nrows; row += stride)  // whole half-warps iterate together
-        merge_row(idx, opart, lpart, out, lse, N, Hq, bs, topk, row);
+        merge_row<VALIDATE>(idx, opart, lpart, out, lse, N, Hq, bs, topk, row);
 }
