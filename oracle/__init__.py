@@ -45,6 +45,8 @@ def _load():
             lib = ctypes.CDLL(_LIB_PATH)
             lib.oracle_pool.restype = None
             lib.oracle_pool.argtypes = [_P, _I, _I, _I, _I, _I, _P]
+            lib.oracle_pool_mode.restype = None
+            lib.oracle_pool_mode.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P]
             lib.oracle_select.restype = None
             lib.oracle_select.argtypes = [_P, _P] + [_I] * 7 + [_P, _I, _P, _P, _P, _P, _I]
             lib.oracle_attend.restype = _I
@@ -75,13 +77,25 @@ def all_rows(B: int, Hq: int, N: int) -> np.ndarray:
     return np.ascontiguousarray(np.stack([b.ravel(), h.ravel(), t.ravel()], axis=1).astype(np.int64))
 
 
-def pool(k: torch.Tensor, block_size: int) -> np.ndarray:
-    """Kbar [B, Hkv, N // block_size, d]: the mean of each full key block, in fp64."""
+POOLINGS = {"mean": 0, "max": 1, "weighted": 2}
+
+
+def pool(k: torch.Tensor, block_size: int, pooling: str = "mean", weights=None) -> np.ndarray:
+    """Kbar [B, Hkv, N // block_size, d] in fp64: the mean of each full key block (default), the
+    feature-wise maximum ("max"), or the weighted mean with one weight per position inside a
+    block ("weighted", weights: block_size non-negative numbers with a positive sum)."""
     _check_bf16(k)
     B, N, Hkv, d = k.shape
     nfull = N // block_size
     kbar = np.zeros((B, Hkv, max(nfull, 1), d), dtype=np.float64)
-    _load().oracle_pool(_ptr(k), B, N, Hkv, d, block_size, _ptr(kbar))
+    mode = POOLINGS[pooling]
+    if mode == 0:
+        _load().oracle_pool(_ptr(k), B, N, Hkv, d, block_size, _ptr(kbar))
+    else:
+        w = np.zeros(1) if weights is None else np.ascontiguousarray(weights, dtype=np.float64)
+        if mode == 2:
+            assert w.shape == (block_size,) and (w >= 0).all() and w.sum() > 0
+        _load().oracle_pool_mode(_ptr(k), B, N, Hkv, d, block_size, mode, _ptr(w), _ptr(kbar))
     return kbar[:, :, :nfull]
 
 
@@ -126,7 +140,8 @@ def attend(q, k, v, block_size: int, topk: int, rows: np.ndarray, sel: np.ndarra
     return out, lse
 
 
-def forward(q, k, v, block_size: int, topk: int, rows: np.ndarray | None = None):
+def forward(q, k, v, block_size: int, topk: int, rows: np.ndarray | None = None, pooling: str = "mean",
+            weights=None):
     """The whole method for the given rows (all rows by default).
 
     Returns a dict with sel, s_last, s_next, out, lse (rows in the order given)."""
@@ -134,7 +149,7 @@ def forward(q, k, v, block_size: int, topk: int, rows: np.ndarray | None = None)
     Hkv = k.shape[2]
     if rows is None:
         rows = all_rows(B, Hq, N)
-    kbar = pool(k, block_size)
+    kbar = pool(k, block_size, pooling, weights)
     sel, s_last, s_next = select(q, kbar, Hkv, block_size, topk, rows)
     out, lse = attend(q, k, v, block_size, topk, rows, sel)
     return {"rows": rows, "sel": sel, "s_last": s_last, "s_next": s_next, "out": out, "lse": lse}

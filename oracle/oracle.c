@@ -15,6 +15,11 @@
  *   2. Mean pooling: the representative of block j is the mean of its keys
  *      (blog "KIMI MoBA", section 3 config field score_pooling = mean, and the
  *      section 4 block-selection simulation that averages each block's keys).
+ *      Variants (the same blog, section 6, suggests trying max pooling or
+ *      weighted pooling instead of the mean): max pooling takes, feature by
+ *      feature, the largest key value of the block; weighted pooling takes
+ *      sum_u w[u - jB] K[u] / sum_p w[p] with one caller-given non-negative
+ *      weight per position inside a block.
  *   3. Parameter-less gating: the score of block j for query q is <q, Kbar_j>,
  *      no learned weights and no scaling ("MoBA project hub", Step 2; tech-
  *      report summary, section 2, relevance score s_i).
@@ -60,6 +65,41 @@ void oracle_pool(const uint16_t* K, int64_t B, int64_t N, int64_t Hkv, int64_t d
                     for (int64_t e = 0; e < d; ++e) dst[e] += bf16_to_double(src[e]);
                 }
                 for (int64_t e = 0; e < d; ++e) dst[e] /= (double)bs;
+            }
+}
+
+/* Step 2, variants. mode 1: Kbar[b, h, j, e] = max over the block's keys of K[u, e].
+ * mode 2: Kbar[b, h, j, :] = sum_p w[p] K[jB + p] / sum_p w[p] (w: bs non-negative weights with a
+ * positive sum). mode 0 is the mean (oracle_pool). */
+void oracle_pool_mode(const uint16_t* K, int64_t B, int64_t N, int64_t Hkv, int64_t d, int64_t bs,
+                      int64_t mode, const double* w, double* Kbar) {
+    if (mode == 0) {
+        oracle_pool(K, B, N, Hkv, d, bs, Kbar);
+        return;
+    }
+    int64_t nfull = N / bs;
+    double wsum = 0.0;
+    if (mode == 2)
+        for (int64_t p = 0; p < bs; ++p) wsum += w[p];
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t h = 0; h < Hkv; ++h)
+            for (int64_t j = 0; j < nfull; ++j) {
+                double* dst = Kbar + ((b * Hkv + h) * nfull + j) * d;
+                for (int64_t e = 0; e < d; ++e) dst[e] = (mode == 1) ? -INFINITY : 0.0;
+                for (int64_t u = j * bs; u < (j + 1) * bs; ++u) {
+                    const uint16_t* src = K + ((b * N + u) * Hkv + h) * d;
+                    for (int64_t e = 0; e < d; ++e) {
+                        double x = bf16_to_double(src[e]);
+                        if (mode == 1) {
+                            if (x > dst[e]) dst[e] = x;
+                        } else {
+                            dst[e] += w[u - j * bs] * x;
+                        }
+                    }
+                }
+                if (mode == 2)
+                    for (int64_t e = 0; e < d; ++e) dst[e] /= wsum;
             }
 }
 
