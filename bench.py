@@ -84,6 +84,8 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-sdpa", action="store_true", help="skip torch's dense attention in the dense arm")
+    p.add_argument("--pooling", choices=("mean", "max", "weighted"), default="mean",
+                   help="the gate's block summary (weighted: weights rising linearly from 0.5 to 1.5 across a block)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--sample-rows", type=int, default=1024, help="oracle rows per CPU sample")
     return p.parse_args(argv)
@@ -106,14 +108,24 @@ def workload(seq_len: int | None = None, hq: int | None = None, hkv: int | None 
 def workload_name(w: dict) -> str:
     cfg = w.get("config", DEFAULT_CONFIG)
     base = CONFIGS[cfg]
+    pooling = w.get("pooling", "mean")
+    suffix = "" if pooling == "mean" else f", {pooling} pooling" + (
+        " (weights 0.5..1.5 across a block)" if pooling == "weighted" else "")
     if cfg == DEFAULT_CONFIG and all(w[k] == WORKLOAD[k] for k in ("N", "Hq", "Hkv")):
-        return WORKLOAD_NAME
+        return WORKLOAD_NAME + suffix
     name = (f"{CONFIG_NAMES[cfg]}: B={w['B']}, Hq={w['Hq']}, Hkv={w['Hkv']}, d={w['d']}, N={w['N']}, "
             f"block_size={w['block_size']}, topk={w['topk']}, causal, bf16, seed {w['seed']}")
     if any(w[k] != base[k] for k in ("Hq", "Hkv")) or (w["N"] != base["N"] and not (
             cfg == 3 and w["N"] in (131072, 524288))):
         name += " (diagnostic override)"
-    return name
+    return name + suffix
+
+
+def pool_weights_host(w: dict):
+    """The weighted-pooling recipe of the bench: one weight per position inside a block, rising
+    linearly from 0.5 (first key) to 1.5 (last key), as fp32."""
+    import numpy as np
+    return np.linspace(0.5, 1.5, w["block_size"]).astype(np.float32)
 
 
 def metric_name(w: dict) -> str:
@@ -255,8 +267,10 @@ def oracle_sample(q, k, v, w: dict, n_rows: int, seed: int) -> tuple[float, floa
     import oracle
     total = w["B"] * w["Hq"] * w["N"]
     rows = oracle.all_rows(w["B"], w["Hq"], w["N"]) if total <= n_rows else sample_rows(w, n_rows, seed)
+    pooling = w.get("pooling", "mean")
+    pw = pool_weights_host(w).astype("float64") if pooling == "weighted" else None
     t0 = time.perf_counter()
-    oracle.forward(q, k, v, w["block_size"], w["topk"], rows)
+    oracle.forward(q, k, v, w["block_size"], w["topk"], rows, pooling=pooling, weights=pw)
     dt = time.perf_counter() - t0
     return dt, rows_useful_flops(w, rows), len(rows)
 
@@ -310,6 +324,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = workload(args.seq_len, args.hq, args.hkv, args.config)
+    w["pooling"] = args.pooling
     q, k, v = host_inputs(w, w["seed"], pin=False)
     for i in range(args.warmup):
         oracle_sample(q, k, v, w, args.sample_rows, 1000 + i)
@@ -406,6 +421,7 @@ def run_moba(args):
 
     moba.lib()
     w = workload(args.seq_len, args.hq, args.hkv, args.config)
+    w["pooling"] = args.pooling
     B, N, Hq, Hkv, d, bs, topk = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], w["block_size"], w["topk"]
     split = world > 1 and partition.can_split(Hq, Hkv, world)
     if split:  # one forward, split by kv-head groups
@@ -429,8 +445,10 @@ def run_moba(args):
     in_bytes = (q.numel() + k.numel() + v.numel()) * 2
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if in_bytes < L2_FLUSH_BELOW else None
 
+    pw = torch.from_numpy(pool_weights_host(w)).to(dev) if args.pooling == "weighted" else None
+
     def step():
-        moba.forward(q, k, v, bs, topk, out=out, lse=lse, workspace=ws)
+        moba.forward(q, k, v, bs, topk, out=out, lse=lse, workspace=ws, pooling=args.pooling, pool_weights=pw)
 
     for _ in range(args.warmup):
         step()

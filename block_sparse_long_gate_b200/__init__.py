@@ -24,14 +24,22 @@ MOBA_OK = 0
 STATUS_NAMES = {
     0: "MOBA_OK", 1: "MOBA_ERR_NULL", 2: "MOBA_ERR_SHAPE", 3: "MOBA_ERR_ALIGN", 4: "MOBA_ERR_UNSUPPORTED",
     5: "MOBA_ERR_CUDA", 6: "MOBA_ERR_OOM", 7: "MOBA_ERR_DEVICE_TIMEOUT", 8: "MOBA_ERR_WORKSPACE",
-    9: "MOBA_ERR_SELECTION",
+    9: "MOBA_ERR_SELECTION", 10: "MOBA_ERR_VALUE",
 }
+POOLINGS = {"mean": 0, "max": 1, "weighted": 2}
+
+
+class Options(ctypes.Structure):
+    """moba_options of include/moba.h."""
+    _fields_ = [("struct_size", ctypes.c_uint32), ("pooling", ctypes.c_int32), ("pool_weights", ctypes.c_void_p),
+                ("full_attention", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 EXPORTED = [
     "moba_status_string", "moba_workspace_size", "moba_forward", "moba_forward_ws", "moba_gate",
     "moba_forward_selected", "moba_forward_selected_ws", "moba_dense_causal", "moba_sync_status",
     "moba_set_attention_impl", "moba_set_gate_impl", "moba_stage_timing", "moba_stage_times",
     "moba_launch_count", "moba_gate_noalloc", "moba_last_error_string", "moba_selftest_wait_timeout",
+    "moba_forward_ex", "moba_gate_ex",
 ]
 STAGES = ("pool", "gate", "invert", "attention", "merge")
 
@@ -98,6 +106,11 @@ def lib():
             L.moba_last_error_string.argtypes = []
             L.moba_selftest_wait_timeout.restype = _I
             L.moba_selftest_wait_timeout.argtypes = [_L, _P]
+            L.moba_forward_ex.restype = _I
+            L.moba_forward_ex.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _L, _I, _I, _I, ctypes.POINTER(Options), _P,
+                                          ctypes.c_size_t, _P]
+            L.moba_gate_ex.restype = _I
+            L.moba_gate_ex.argtypes = [_P, _P, _P, _I, _I, _I, _L, _I, _I, _I, ctypes.POINTER(Options), _P]
             L.moba_gate_noalloc.restype = _I
             L.moba_gate_noalloc.argtypes = [_P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P]
             _lib = L
@@ -146,11 +159,41 @@ def workspace_size(B, Hq, Hkv, N, d, block_size, topk) -> int:
     return int(n.value)
 
 
-def forward(q, k, v, block_size: int, topk: int, out=None, lse=None, workspace=None, stream=None):
-    """MoBA causal prefill forward. Returns (out bf16 [B, N, Hq, d], lse fp32 [B, Hq, N])."""
+def options(pooling: str = "mean", pool_weights=None, full_attention: bool = False) -> Options:
+    """moba_options for the extended entry points. pool_weights: fp32 CUDA tensor [block_size]."""
+    if pooling not in POOLINGS:
+        raise ValueError(f"pooling must be one of {sorted(POOLINGS)}")
+    if pool_weights is not None and (pool_weights.dtype != torch.float32 or not pool_weights.is_cuda
+                                     or not pool_weights.is_contiguous()):
+        raise ValueError("pool_weights must be a contiguous fp32 CUDA tensor")
+    o = Options()
+    o.struct_size = ctypes.sizeof(Options)
+    o.pooling = POOLINGS[pooling]
+    o.pool_weights = _ptr(pool_weights)
+    o.full_attention = 1 if full_attention else 0
+    o.reserved = 0
+    return o
+
+
+def forward(q, k, v, block_size: int, topk: int, out=None, lse=None, workspace=None, stream=None,
+            pooling: str = "mean", pool_weights=None, full_attention: bool = False):
+    """MoBA causal prefill forward. Returns (out bf16 [B, N, Hq, d], lse fp32 [B, Hq, N]).
+
+    pooling / pool_weights choose the gate's block summary ("mean", "max", "weighted"), and
+    full_attention=True makes this a full-attention layer of a hybrid model (dense causal)."""
     B, N, Hq, Hkv, d = _check_qkv(q, k, v)
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    if pooling != "mean" or full_attention:
+        opt = options(pooling, pool_weights, full_attention)
+        if workspace is None and not full_attention:
+            workspace = torch.empty(workspace_size(B, Hq, Hkv, N, d, block_size, topk), dtype=torch.uint8,
+                                    device=q.device)
+        _check(lib().moba_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d, block_size,
+                                     topk, ctypes.byref(opt), _ptr(workspace),
+                                     0 if workspace is None else workspace.numel(), _stream(stream)),
+               "moba_forward_ex")
+        return out, lse
     if workspace is None:
         workspace = torch.empty(workspace_size(B, Hq, Hkv, N, d, block_size, topk), dtype=torch.uint8,
                                 device=q.device)
@@ -159,10 +202,15 @@ def forward(q, k, v, block_size: int, topk: int, out=None, lse=None, workspace=N
     return out, lse
 
 
-def gate(q, k, block_size: int, topk: int, idx=None, stream=None):
+def gate(q, k, block_size: int, topk: int, idx=None, stream=None, pooling: str = "mean", pool_weights=None):
     """Selected blocks per query: int32 [B, Hq, N, topk], ascending, own block last, -1 padded."""
     B, N, Hq, Hkv, d = _check_qkv(q, k)
     idx = torch.empty((B, Hq, N, topk), dtype=torch.int32, device=q.device) if idx is None else idx
+    if pooling != "mean":
+        opt = options(pooling, pool_weights)
+        _check(lib().moba_gate_ex(_ptr(q), _ptr(k), _ptr(idx), B, Hq, Hkv, N, d, block_size, topk, ctypes.byref(opt),
+                                  _stream(stream)), "moba_gate_ex")
+        return idx
     _check(lib().moba_gate(_ptr(q), _ptr(k), _ptr(idx), B, Hq, Hkv, N, d, block_size, topk, _stream(stream)),
            "moba_gate")
     return idx

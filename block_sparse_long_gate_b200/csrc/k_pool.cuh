@@ -10,6 +10,11 @@
 // mean carries a single rounding (the division) and the gate sees the same
 // block representatives as an exact evaluation would.
 //
+// Variants ("KIMI MoBA" blog, section 6: try max or weighted pooling): the
+// feature-wise maximum over the block's keys (exact), or the weighted mean
+// sum_p w[p] K[jB + p] / sum_p w[p] with one fp32 weight per position inside a
+// block (products and sums in double).
+//
 // Streaming reduction, HBM bound: 2 * block_size * d bytes read per (b, h, j).
 #pragma once
 #include "common.cuh"
@@ -29,10 +34,17 @@ struct PoolAux {
     unsigned* head_stats;   // [B*Hkv][2], zeroed before the launch
 };
 
+// Pooling of a block: 0 mean, 1 feature-wise max, 2 weighted mean with weights w[0, bs).
+struct PoolMode {
+    int mode;
+    const float* w;
+};
+
 // grid (nfull, Hkv, B); 16 row groups x 16 threads that each read 16 bytes.
 __global__ void __launch_bounds__(POOL_THREADS) moba_pool_kernel(const uint16_t* __restrict__ K,
                                                                  double* __restrict__ kbar, int64_t N,
-                                                                 int Hkv, int bs, int64_t nfull, PoolAux aux) {
+                                                                 int Hkv, int bs, int64_t nfull, PoolAux aux,
+                                                                 PoolMode pm) {
     const int64_t j = blockIdx.x;
     const int h = blockIdx.y, b = blockIdx.z;
     const int c16 = threadIdx.x & 15;
@@ -40,20 +52,22 @@ __global__ void __launch_bounds__(POOL_THREADS) moba_pool_kernel(const uint16_t*
     const int64_t rstride = (int64_t)Hkv * MOBA_D;
     const uint16_t* base = K + (((int64_t)b * N + j * bs) * Hkv + h) * MOBA_D + c16 * 8;
 
+    const bool is_max = pm.mode == 1, is_w = pm.mode == 2;
     double acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+    for (int i = 0; i < 8; ++i) acc[i] = is_max ? -INFINITY : 0.0;
 
-    auto add = [&](const uint4& w) {
-        acc[0] += (double)bf16lo(w.x);
-        acc[1] += (double)bf16hi(w.x);
-        acc[2] += (double)bf16lo(w.y);
-        acc[3] += (double)bf16hi(w.y);
-        acc[4] += (double)bf16lo(w.z);
-        acc[5] += (double)bf16hi(w.z);
-        acc[6] += (double)bf16lo(w.w);
-        acc[7] += (double)bf16hi(w.w);
+    auto add = [&](const uint4& w, double wt) {
+        const float f[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
+                            bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (is_max) acc[i] = fmax(acc[i], (double)f[i]);
+            else if (is_w) acc[i] = fma(wt, (double)f[i], acc[i]);
+            else acc[i] += (double)f[i];
+        }
     };
+    auto wt_at = [&](int u) { return is_w ? (double)__ldg(pm.w + u) : 1.0; };
 
     int u = rg;
     for (; u + 48 < bs; u += 64) {
@@ -61,23 +75,50 @@ __global__ void __launch_bounds__(POOL_THREADS) moba_pool_kernel(const uint16_t*
         uint4 w1 = ld_nc_v4(base + (int64_t)(u + 16) * rstride);
         uint4 w2 = ld_nc_v4(base + (int64_t)(u + 32) * rstride);
         uint4 w3 = ld_nc_v4(base + (int64_t)(u + 48) * rstride);
-        add(w0);
-        add(w1);
-        add(w2);
-        add(w3);
+        add(w0, wt_at(u));
+        add(w1, wt_at(u + 16));
+        add(w2, wt_at(u + 32));
+        add(w3, wt_at(u + 48));
     }
-    for (; u < bs; u += 16) add(ld_nc_v4(base + (int64_t)u * rstride));
+    for (; u < bs; u += 16) add(ld_nc_v4(base + (int64_t)u * rstride), wt_at(u));
 
     __shared__ double red[16][MOBA_D];
+    __shared__ double wred[POOL_THREADS / 32];
+    __shared__ int wbad;
 #pragma unroll
     for (int i = 0; i < 8; ++i) red[rg][c16 * 8 + i] = acc[i];
+    double wsum = (double)bs;
+    if (is_w) {  // sum of the weights (and a check that none is negative)
+        double sw = 0.0;
+        int bad = 0;
+        for (int p = threadIdx.x; p < bs; p += POOL_THREADS) {
+            const float wp = __ldg(pm.w + p);
+            sw += (double)wp;
+            bad |= !(wp >= 0.f);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sw += __shfl_xor_sync(0xffffffffu, sw, o);
+        bad = __any_sync(0xffffffffu, bad);
+        if (threadIdx.x == 0) wbad = 0;
+        __syncthreads();
+        if ((threadIdx.x & 31) == 0) {
+            wred[threadIdx.x >> 5] = sw;
+            if (bad) wbad = 1;
+        }
+    }
     __syncthreads();
+    if (is_w) {
+        wsum = 0.0;
+#pragma unroll
+        for (int i = 0; i < POOL_THREADS / 32; ++i) wsum += wred[i];
+        if (threadIdx.x == 0 && (wbad || !(wsum > 0.0))) moba_set_error(MOBA_ERR_VALUE);
+    }
     double x = 0.0;
     if (threadIdx.x < MOBA_D) {
-        double s = 0.0;
+        double s = is_max ? -INFINITY : 0.0;
 #pragma unroll
-        for (int g = 0; g < 16; ++g) s += red[g][threadIdx.x];
-        x = s / (double)bs;
+        for (int g = 0; g < 16; ++g) s = is_max ? fmax(s, red[g][threadIdx.x]) : s + red[g][threadIdx.x];
+        x = is_max ? s : s / wsum;
         kbar[(((int64_t)b * Hkv + h) * nfull + j) * MOBA_D + threadIdx.x] = x;
     }
     if (aux.planes == nullptr) return;

@@ -213,7 +213,7 @@ GateScratch gate_scratch(const Plan& P, char* ws, bool tc) {
 
 bool use_tc_gate(const Plan& P) { return g_gate_impl.load() == 0 && P.nfull > 0 && P.kp > 0; }
 
-int run_pool(const Plan& P, const void* k, const GateScratch& gs, cudaStream_t st) {
+int run_pool(const Plan& P, const void* k, const GateScratch& gs, PoolMode pm, cudaStream_t st) {
     if (P.nfull == 0) return MOBA_OK;
     if (gs.aux.head_stats) {
         const cudaError_t e = cudaMemsetAsync(gs.aux.head_stats, 0, sizeof(unsigned) * 2 * (size_t)P.B * P.Hkv, st);
@@ -221,7 +221,7 @@ int run_pool(const Plan& P, const void* k, const GateScratch& gs, cudaStream_t s
     }
     dim3 grid((unsigned)P.nfull, P.Hkv, P.B);
     moba_pool_kernel<<<grid, POOL_THREADS, 0, st>>>((const uint16_t*)k, gs.kbar, P.N, P.Hkv, P.bs, P.nfull,
-                                                    gs.aux);
+                                                    gs.aux, pm);
     count_launch();
     return launch_ok();
 }
@@ -392,7 +392,7 @@ int run_merge(const Plan& P, const int32_t* idx, bool validate, char* ws, void* 
 
 int forward_impl(const void* q, const void* k, const void* v, const int32_t* idx_in, void* out, float* lse,
                  int B, int Hq, int Hkv, int64_t N, int d, int bs, int topk, void* ws_ptr, size_t ws_bytes,
-                 cudaStream_t st) {
+                 cudaStream_t st, PoolMode pm = PoolMode{0, nullptr}) {
     Plan P;
     int rc = make_plan(B, Hq, Hkv, N, d, bs, topk, &P);
     if (rc) return rc;
@@ -417,7 +417,7 @@ int forward_impl(const void* q, const void* k, const void* v, const int32_t* idx
         if (!idx) {
             int32_t* widx = (int32_t*)(ws + P.off_idx);
             const GateScratch gs = gate_scratch(P, ws, use_tc_gate(P));
-            if ((rc = run_pool(P, k, gs, st))) break;
+            if ((rc = run_pool(P, k, gs, pm, st))) break;
             timer.mark(done++);
             if ((rc = run_gate(P, q, gs, widx, st))) break;
             timer.mark(done++);
@@ -439,6 +439,36 @@ int forward_impl(const void* q, const void* k, const void* v, const int32_t* idx
     return rc;
 }
 
+// Options of the extended entry points; NULL means the defaults.
+int parse_options(const moba_options* o, PoolMode* pm, bool* full) {
+    *pm = PoolMode{0, nullptr};
+    *full = false;
+    if (!o) return MOBA_OK;
+    if (o->struct_size < sizeof(moba_options) || o->reserved != 0) return MOBA_ERR_SHAPE;
+    if (o->pooling < MOBA_POOL_MEAN || o->pooling > MOBA_POOL_WEIGHTED) return MOBA_ERR_SHAPE;
+    if (o->pooling == MOBA_POOL_WEIGHTED && (!o->pool_weights || !aligned16(o->pool_weights))) return MOBA_ERR_SHAPE;
+    if (o->full_attention != 0 && o->full_attention != 1) return MOBA_ERR_SHAPE;
+    pm->mode = o->pooling;
+    pm->w = o->pooling == MOBA_POOL_WEIGHTED ? o->pool_weights : nullptr;
+    *full = o->full_attention == 1;
+    return MOBA_OK;
+}
+
+int dense_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int64_t N,
+               int d, cudaStream_t st) {
+    Plan P;
+    if (N < 1 || N >= ((int64_t)1 << 31)) return MOBA_ERR_SHAPE;
+    int rc = make_plan(B, Hq, Hkv, N, d, (int)N, 1, &P);
+    if (rc) return rc;
+    if ((rc = check_ptrs({q, k, v, out, lse}))) return rc;
+    if ((rc = check_device())) return rc;
+    AttnParams a = attn_params(P, q, k, v, out, lse, nullptr);
+    a.dense = 1;
+    a.Pmax = 0;
+    a.L = 0;
+    return run_attention(P, a, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -455,6 +485,7 @@ const char* moba_status_string(int s) {
         case MOBA_ERR_DEVICE_TIMEOUT: return "device wait reached its limit";
         case MOBA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
         case MOBA_ERR_SELECTION: return "malformed selection row";
+        case MOBA_ERR_VALUE: return "invalid argument values (pooling weights)";
         default: return "unknown status";
     }
 }
@@ -513,7 +544,7 @@ int moba_gate(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv
         return MOBA_ERR_OOM;
     }
     const GateScratch gs = gate_scratch(P, scratch, use_tc_gate(P));
-    rc = run_pool(P, k, gs, st);
+    rc = run_pool(P, k, gs, PoolMode{0, nullptr}, st);
     if (!rc) rc = run_gate(P, q, gs, idx, st);
     cudaFreeAsync(scratch, st);
     return rc;
@@ -521,17 +552,47 @@ int moba_gate(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv
 
 int moba_dense_causal(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
                       int64_t N, int d, moba_stream_t stream) {
-    Plan P;
-    if (N < 1 || N >= ((int64_t)1 << 31)) return MOBA_ERR_SHAPE;
-    int rc = make_plan(B, Hq, Hkv, N, d, (int)N, 1, &P);
+    return dense_impl(q, k, v, out, lse, B, Hq, Hkv, N, d, (cudaStream_t)stream);
+}
+
+int moba_forward_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                    int64_t N, int d, int block_size, int topk, const moba_options* options, void* workspace,
+                    size_t workspace_bytes, moba_stream_t stream) {
+    PoolMode pm;
+    bool full = false;
+    int rc = parse_options(options, &pm, &full);
     if (rc) return rc;
-    if ((rc = check_ptrs({q, k, v, out, lse}))) return rc;
+    if (full) {  // a full-attention layer of a hybrid model
+        Plan P;
+        if ((rc = make_plan(B, Hq, Hkv, N, d, block_size, topk, &P))) return rc;
+        return dense_impl(q, k, v, out, lse, B, Hq, Hkv, N, d, (cudaStream_t)stream);
+    }
+    return forward_impl(q, k, v, nullptr, out, lse, B, Hq, Hkv, N, d, block_size, topk, workspace, workspace_bytes,
+                        (cudaStream_t)stream, pm);
+}
+
+int moba_gate_ex(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv, int64_t N, int d,
+                 int block_size, int topk, const moba_options* options, moba_stream_t stream) {
+    PoolMode pm;
+    bool full = false;
+    int rc = parse_options(options, &pm, &full);
+    if (rc) return rc;
+    if (full) return MOBA_ERR_SHAPE;  // a full-attention layer has no gate
+    Plan P;
+    if ((rc = make_plan(B, Hq, Hkv, N, d, block_size, topk, &P))) return rc;
+    if ((rc = check_ptrs({q, k, (const void*)idx}))) return rc;
     if ((rc = check_device())) return rc;
-    AttnParams a = attn_params(P, q, k, v, out, lse, nullptr);
-    a.dense = 1;
-    a.Pmax = 0;
-    a.L = 0;
-    return run_attention(P, a, (cudaStream_t)stream);
+    cudaStream_t st = (cudaStream_t)stream;
+    char* scratch = nullptr;
+    if (cudaMallocAsync((void**)&scratch, P.gate_bytes, st) != cudaSuccess) {
+        cudaGetLastError();
+        return MOBA_ERR_OOM;
+    }
+    const GateScratch gs = gate_scratch(P, scratch, use_tc_gate(P));
+    rc = run_pool(P, k, gs, pm, st);
+    if (!rc) rc = run_gate(P, q, gs, idx, st);
+    cudaFreeAsync(scratch, st);
+    return rc;
 }
 
 int moba_sync_status(moba_stream_t stream) {
@@ -693,7 +754,7 @@ extern "C" int moba_gate_noalloc(const void* q, const void* k, int32_t* idx, int
     GateScratch gs;
     gs.kbar = kbar;
     gs.aux = PoolAux{nullptr, nullptr, nullptr};  // the fp64 gate: its only scratch is Kbar
-    rc = run_pool(P, k, gs, st);
+    rc = run_pool(P, k, gs, PoolMode{0, nullptr}, st);
     if (!rc) rc = run_gate(P, q, gs, idx, st);
     return rc;
 }

@@ -59,8 +59,30 @@ typedef enum {
     MOBA_ERR_OOM = 6,            /* the internal workspace could not be allocated */
     MOBA_ERR_DEVICE_TIMEOUT = 7, /* a kernel gave up waiting (bounded wait hit its limit) */
     MOBA_ERR_WORKSPACE = 8,      /* the caller's workspace is NULL or too small */
-    MOBA_ERR_SELECTION = 9       /* an injected selection is malformed (found on the device) */
+    MOBA_ERR_SELECTION = 9,      /* an injected selection is malformed (found on the device) */
+    MOBA_ERR_VALUE = 10          /* an argument's values are invalid (found on the device): pooling weights */
 } moba_status;
+
+/* How a key block is summarised for the gate ("KIMI MoBA" blog: section 3 field
+ * score_pooling = mean; section 6 suggests max or weighted pooling instead). */
+typedef enum {
+    MOBA_POOL_MEAN = 0,     /* mean of the block's keys (the method's default) */
+    MOBA_POOL_MAX = 1,      /* feature-wise maximum over the block's keys */
+    MOBA_POOL_WEIGHTED = 2  /* sum_p w[p] K[jB + p] / sum_p w[p], one weight per position in a block */
+} moba_pooling;
+
+/* Options of the extended entry points (moba_forward_ex, moba_gate_ex). Zero-initialise,
+ * set struct_size = sizeof(moba_options), then the fields wanted; a NULL options pointer means
+ * all defaults (mean pooling, MoBA attention). */
+typedef struct moba_options {
+    uint32_t struct_size;       /* sizeof(moba_options) */
+    int32_t pooling;            /* moba_pooling */
+    const float* pool_weights;  /* MOBA_POOL_WEIGHTED: DEVICE fp32 [block_size], every w >= 0 with a
+                                   positive sum (checked on the device: MOBA_ERR_VALUE); else NULL */
+    int32_t full_attention;     /* hybrid-layer switch ("KIMI MoBA" blog, section 3, hybrid_layers):
+                                   1 = this layer uses full causal attention (no gating); 0 = MoBA */
+    int32_t reserved;           /* must be 0 */
+} moba_options;
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* moba_status_string(int status);
@@ -95,6 +117,18 @@ int moba_forward_ws(const void* q, const void* k, const void* v, void* out, floa
                     size_t workspace_bytes, moba_stream_t stream);
 
 /*
+ * moba_forward_ws with options: the gate's pooling (mean, max, weighted) and the hybrid-layer
+ * switch (full_attention = 1 runs dense causal attention, as moba_dense_causal, and needs no
+ * workspace). A NULL workspace is allocated with cudaMallocAsync on `stream`, as moba_forward
+ * does. Same layouts, ownership and errors as moba_forward_ws;
+ * MOBA_ERR_SHAPE for an unknown pooling, a NULL pool_weights with MOBA_POOL_WEIGHTED, a
+ * struct_size below sizeof(moba_options) or reserved != 0.
+ */
+int moba_forward_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                    int Hkv, int64_t N, int d, int block_size, int topk, const moba_options* options,
+                    void* workspace, size_t workspace_bytes, moba_stream_t stream);
+
+/*
  * Gating only: block mean pooling, scores <q_t, Kbar_j> over earlier blocks,
  * forced own block and top-k. Writes idx (int32 [B, Hq, N, topk]).
  * Defined by: "MoBA project hub" page, Step 2 (score of a block = inner product
@@ -106,6 +140,11 @@ int moba_forward_ws(const void* q, const void* k, const void* v, void* out, floa
  */
 int moba_gate(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv, int64_t N, int d,
               int block_size, int topk, moba_stream_t stream);
+
+/* moba_gate with options (the pooling; full_attention must be 0). Allocates its scratch with
+ * cudaMallocAsync on `stream`. */
+int moba_gate_ex(const void* q, const void* k, int32_t* idx, int B, int Hq, int Hkv, int64_t N, int d,
+                 int block_size, int topk, const moba_options* options, moba_stream_t stream);
 
 /*
  * Attention with a given selection idx (same layout as moba_gate's output):

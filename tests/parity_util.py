@@ -80,11 +80,12 @@ class SelectionReport:
         return self
 
 
-def check_selection_all_rows(idx_dev, q_h, k_h, Hkv, bs, topk, what, exact_ties_strict=False):
+def check_selection_all_rows(idx_dev, q_h, k_h, Hkv, bs, topk, what, exact_ties_strict=False, pooling="mean",
+                             weights=None):
     """Every row of the device selection idx [B, Hq, N, topk] against the oracle, one head
-    at a time (the oracle pools K once)."""
+    at a time (the oracle pools K once, with the given pooling)."""
     B, N, Hq, _ = q_h.shape
-    kbar = oracle.pool(k_h, bs)
+    kbar = oracle.pool(k_h, bs, pooling, weights)
     rep = SelectionReport(what + " (all rows)")
     t = np.arange(N, dtype=np.int64)
     for b in range(B):

@@ -26,7 +26,7 @@ def test_every_declared_symbol_is_exported(moba):
 
 def test_status_strings(moba):
     L = moba.lib()
-    for s in range(10):
+    for s in range(11):
         assert L.moba_status_string(s).decode() not in ("", "unknown status")
     assert L.moba_status_string(99).decode() == "unknown status"
 
