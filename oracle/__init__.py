@@ -155,6 +155,35 @@ def forward(q, k, v, block_size: int, topk: int, rows: np.ndarray | None = None,
     return {"rows": rows, "sel": sel, "s_last": s_last, "s_next": s_next, "out": out, "lse": lse}
 
 
+def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_size: int, topk: int, length: int,
+           pooling: str = "mean", weights=None, full_attention: bool = False):
+    """One decode step: the query q [B, Hq, d] is the token at position length - 1 of each sequence,
+    attending its KV cache k, v [B, >= length, Hkv, d] (keys 0 .. length - 1). It is the prefill
+    definition at that row (the gate, its causal rules and the attention of the pages), so the oracle
+    evaluates row length - 1 of a prefill whose query tensor holds q there. full_attention: every
+    earlier block is kept (the full-attention decode of a hybrid model).
+
+    Returns a dict with sel [B * Hq, topk], s_last, s_next, out [B * Hq, d], lse [B * Hq]
+    (rows b-major, then head)."""
+    _check_bf16(k, v)
+    B, Hq, d = q.shape
+    Hkv = k.shape[2]
+    L = int(length)
+    kk = k[:, :L].contiguous()
+    vv = v[:, :L].contiguous()
+    qf = torch.zeros((B, L, Hq, d), dtype=torch.bfloat16)
+    qf[:, L - 1] = q
+    rows = np.ascontiguousarray(np.stack(np.meshgrid(np.arange(B), np.arange(Hq), indexing="ij"), -1)
+                                .reshape(-1, 2))
+    rows = np.ascontiguousarray(np.concatenate([rows, np.full((len(rows), 1), L - 1)], 1).astype(np.int64))
+    nblk = (L + block_size - 1) // block_size
+    kk_top = nblk if full_attention else topk
+    kbar = pool(kk, block_size, pooling, weights)
+    sel, s_last, s_next = select(qf, kbar, Hkv, block_size, kk_top, rows)
+    out, lse = attend(qf, kk, vv, block_size, kk_top, rows, sel)
+    return {"rows": rows, "sel": sel, "s_last": s_last, "s_next": s_next, "out": out, "lse": lse}
+
+
 def near_tie(s_last: np.ndarray, s_next: np.ndarray, rel: float = 1e-5) -> np.ndarray:
     """Rows whose boundary is a near tie: the last selected and the first unselected past
     scores differ by less than `rel` relative to the larger magnitude of the two,
