@@ -84,6 +84,8 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-sdpa", action="store_true", help="skip torch's dense attention in the dense arm")
+    p.add_argument("--mode", choices=("prefill", "decode"), default="prefill",
+                   help="decode: one new query per sequence against a KV cache of the workload's length")
     p.add_argument("--pooling", choices=("mean", "max", "weighted"), default="mean",
                    help="the gate's block summary (weighted: weights rising linearly from 0.5 to 1.5 across a block)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -600,10 +602,141 @@ def run_moba(args):
     return 0
 
 
+def decode_bytes(B, Hq, Hkv, L, d, bs, topk, idx_host, full: bool) -> tuple[float, int]:
+    """Algorithmic HBM bytes of one decode step: K and V of the blocks the step reads (the union of
+    the kept blocks of each kv head's query heads, the own block up to L - 1), the block summaries
+    the gate reads (fp64, c rows per kv head), q in and out / lse written. Also the number of
+    blocks read."""
+    c = (L - 1) // bs
+    G = Hq // Hkv
+    blocks = 0
+    keys = 0
+    for b in range(B):
+        for hk in range(Hkv):
+            if full:
+                kept = set(range(c + 1))
+            else:
+                kept = {int(j) for h in range(hk * G, (hk + 1) * G) for j in idx_host[b, h] if j >= 0}
+            blocks += len(kept)
+            keys += sum((L - j * bs) if j == c else bs for j in kept)
+    kv = keys * 2 * d * 2
+    gate = 0 if full else B * Hkv * c * d * 8
+    return float(kv + gate + B * Hq * d * 2 * 2 + B * Hq * 4), blocks
+
+
+def run_decode(args):
+    """One decode step per sequence: the newest query of each of the workload's sequences against
+    a KV cache holding the workload's length (all sequences of the batch the same length)."""
+    import torch
+
+    from block_sparse_long_gate_b200.build import build_library
+    build_library()
+    import block_sparse_long_gate_b200 as moba
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        raise SystemExit("--mode decode runs on one GPU")
+    dev = torch.device("cuda", 0)
+    w = workload(args.seq_len, args.hq, args.hkv, args.config)
+    B, L, Hq, Hkv, d, bs, topk = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], w["block_size"], w["topk"]
+    _, k_h, v_h = synth.inputs(B, L, 1, Hkv, d, bs, w["seed"], pin=True)
+    q_h = synth.normal(w["seed"] + 1000, synth.Q_ID, (B, Hq, d), pin=True)
+    k, v, q = k_h.to(dev), v_h.to(dev), q_h.to(dev)
+    del k_h, v_h
+    kbar = moba.pool_cache(k, bs, L)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, Hq, topk), dtype=torch.int32, device=dev)
+    res = {}
+    stream = torch.cuda.current_stream()
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else "0"
+    peaks, peak_src = read_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    clocks = None
+    for full in (False, True):
+        ws = torch.empty(moba.decode_workspace_size(B, Hq, Hkv, L, d, bs, topk, full), dtype=torch.uint8, device=dev)
+
+        def step():
+            moba.decode(q, k, v, kbar, bs, topk, L, full_attention=full, out=out, lse=lse,
+                        idx=None if full else idx, workspace=ws)
+
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize()
+        n = max(args.steps, 20)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        l0 = moba.launch_count()
+        with ClockSampler(gpu_id) as clk:
+            for a, b_ in ev:
+                flush.fill_(1)  # the cache is re-read from HBM, not L2, every step
+                a.record(stream)
+                step()
+                b_.record(stream)
+            torch.cuda.synchronize()
+        launches = (moba.launch_count() - l0) // n
+        us = statistics.median(a.elapsed_time(b_) for a, b_ in ev) * 1e3
+        status = moba.sync_status()
+        nbytes, blocks = decode_bytes(B, Hq, Hkv, L, d, bs, topk, None if full else idx.cpu().numpy(), full)
+        res["full" if full else "moba"] = {"us": us, "bytes": nbytes, "blocks_read": blocks,
+                                           "achieved_gbs": nbytes / (us * 1e-6) / 1e9, "launches": launches,
+                                           "status": status}
+        if not full:
+            clocks = clk.summary()
+        del ws
+    sd = None
+    if not args.no_sdpa:  # torch's fused attention of the single query over the whole cache
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        qt = q.unsqueeze(2)
+        kt, vt = k.permute(0, 2, 1, 3), v.permute(0, 2, 1, 3)
+        try:
+            with sdpa_kernel([SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION]):
+                for _ in range(3):
+                    torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, enable_gqa=Hq != Hkv)
+                torch.cuda.synchronize()
+                ts = []
+                for _ in range(10):
+                    flush.fill_(1)
+                    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, enable_gqa=Hq != Hkv)
+                    b_.record(stream)
+                    torch.cuda.synchronize()
+                    ts.append(a.elapsed_time(b_) * 1e3)
+            sd = {"us": statistics.median(ts), "kernel": "torch sdpa"}
+        except RuntimeError as exc:
+            sd = {"error": str(exc).splitlines()[0][:200]}
+    m = res["moba"]
+    line = {
+        "metric": "MoBA decode step latency (one new token per sequence)", "value": m["us"], "unit": "us",
+        "n_gpus": 1, "steps": max(args.steps, 20), "warmup": max(args.warmup, 3), "ms_per_step": m["us"] / 1e3,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "decode step, KV cache of " + workload_name(w), "global_batch": B, "seq_len": L,
+                   "parallelism": "single GPU", "l2": "a 256 MB buffer is rewritten before every timed step"},
+        "tokens_per_s": B / (m["us"] * 1e-6),
+        "roofline": {"kernel": "moba decode (select + attend + merge)", "bound": "hbm", "achieved": m["achieved_gbs"],
+                     "peak": hbm, "unit": "GB/s", "frac": m["achieved_gbs"] / hbm, "traffic": None,
+                     "bytes_per_step": m["bytes"], "peak_source": f"hbm_gbs of {peak_src}"},
+        "full_attention_decode": res["full"],
+        "speedup_vs_full_attention_decode": res["full"]["us"] / m["us"],
+        "torch_sdpa_decode": sd,
+        "gpu_launches": m["launches"], "clocks": clocks, "device_status": m["status"],
+        "blocks_read": m["blocks_read"],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.mode == "decode":
+        return run_decode(args)
     return run_moba(args)
 
 

@@ -39,7 +39,7 @@ EXPORTED = [
     "moba_forward_selected", "moba_forward_selected_ws", "moba_dense_causal", "moba_sync_status",
     "moba_set_attention_impl", "moba_set_gate_impl", "moba_stage_timing", "moba_stage_times",
     "moba_launch_count", "moba_gate_noalloc", "moba_last_error_string", "moba_selftest_wait_timeout",
-    "moba_forward_ex", "moba_gate_ex",
+    "moba_forward_ex", "moba_gate_ex", "moba_decode_workspace_size", "moba_pool_cache", "moba_decode",
 ]
 STAGES = ("pool", "gate", "invert", "attention", "merge")
 
@@ -111,6 +111,13 @@ def lib():
                                           ctypes.c_size_t, _P]
             L.moba_gate_ex.restype = _I
             L.moba_gate_ex.argtypes = [_P, _P, _P, _I, _I, _I, _L, _I, _I, _I, ctypes.POINTER(Options), _P]
+            L.moba_decode_workspace_size.restype = _I
+            L.moba_decode_workspace_size.argtypes = [_I, _I, _I, _L, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]
+            L.moba_pool_cache.restype = _I
+            L.moba_pool_cache.argtypes = [_P, _P, _I, _I, _L, _L, _I, _I, _L, _L, ctypes.POINTER(Options), _P]
+            L.moba_decode.restype = _I
+            L.moba_decode.argtypes = [_P, _P, _P, _P, _L, _P, _P, _P, _I, _I, _I, _L, _L, _I, _I, _I, _I, _P,
+                                      ctypes.c_size_t, _P]
             L.moba_gate_noalloc.restype = _I
             L.moba_gate_noalloc.argtypes = [_P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P]
             _lib = L
@@ -242,6 +249,52 @@ def forward_selected(q, k, v, idx, block_size: int, topk: int, out=None, lse=Non
                                           N, d, block_size, topk, _ptr(workspace), workspace.numel(),
                                           _stream(stream)), "moba_forward_selected_ws")
     return out, lse
+
+
+def decode_workspace_size(B, Hq, Hkv, L, d, block_size, topk, full_attention=False) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moba_decode_workspace_size(B, Hq, Hkv, L, d, block_size, topk, 1 if full_attention else 0,
+                                            ctypes.byref(n)), "moba_decode_workspace_size")
+    return int(n.value)
+
+
+def pool_cache(k, block_size: int, length: int, kbar=None, first_block: int = 0, pooling: str = "mean",
+               pool_weights=None, stream=None):
+    """Block summaries (fp64 [B, Hkv, rows, d]) of the full blocks of a KV cache k [B, Lmax, Hkv, d]
+    holding `length` tokens; blocks before first_block are left as they are in `kbar`."""
+    if k.dtype != torch.bfloat16 or not k.is_cuda or not k.is_contiguous() or k.dim() != 4:
+        raise ValueError("k must be a contiguous bf16 CUDA tensor [B, Lmax, Hkv, d]")
+    B, Lmax, Hkv, d = k.shape
+    rows = max(length // block_size, 1)
+    if kbar is None:
+        kbar = torch.zeros((B, Hkv, rows, d), dtype=torch.float64, device=k.device)
+    opt = options(pooling, pool_weights)
+    _check(lib().moba_pool_cache(_ptr(k), _ptr(kbar), B, Hkv, length, Lmax, d, block_size, kbar.shape[2],
+                                 first_block, ctypes.byref(opt), _stream(stream)), "moba_pool_cache")
+    return kbar
+
+
+def decode(q, k, v, kbar, block_size: int, topk: int, length: int, full_attention: bool = False, out=None,
+           lse=None, idx=None, workspace=None, stream=None):
+    """One decode step: q [B, Hq, d] (the token at position length - 1) against the cache k, v
+    [B, Lmax, Hkv, d]. Returns (out [B, Hq, d], lse [B, Hq], idx [B, Hq, topk] or None)."""
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    B, Hq, d = q.shape
+    _, Lmax, Hkv, _ = k.shape
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
+    if idx is None and not full_attention:
+        idx = torch.empty((B, Hq, topk), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_size(B, Hq, Hkv, length, d, block_size, topk, full_attention),
+                                dtype=torch.uint8, device=q.device)
+    rows = 0 if kbar is None else kbar.shape[2]
+    _check(lib().moba_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(kbar), rows, _ptr(out), _ptr(lse), _ptr(idx), B, Hq,
+                             Hkv, length, Lmax, d, block_size, topk, 1 if full_attention else 0, _ptr(workspace),
+                             workspace.numel(), _stream(stream)), "moba_decode")
+    return out, lse, idx
 
 
 def dense_causal(q, k, v, out=None, lse=None, stream=None):

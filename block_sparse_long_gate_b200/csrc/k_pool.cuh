@@ -35,9 +35,13 @@ struct PoolAux {
 };
 
 // Pooling of a block: 0 mean, 1 feature-wise max, 2 weighted mean with weights w[0, bs).
+// j0 / rows: the grid pools blocks j0 + blockIdx.x into rows of a summary buffer with `rows`
+// rows per (b, kv head) (a KV cache pools only the blocks that became full; rows = 0 means nfull).
 struct PoolMode {
     int mode;
     const float* w;
+    int64_t j0 = 0;
+    int64_t rows = 0;
 };
 
 // grid (nfull, Hkv, B); 16 row groups x 16 threads that each read 16 bytes.
@@ -45,7 +49,8 @@ __global__ void __launch_bounds__(POOL_THREADS) moba_pool_kernel(const uint16_t*
                                                                  double* __restrict__ kbar, int64_t N,
                                                                  int Hkv, int bs, int64_t nfull, PoolAux aux,
                                                                  PoolMode pm) {
-    const int64_t j = blockIdx.x;
+    const int64_t j = pm.j0 + blockIdx.x;
+    const int64_t krows = pm.rows > 0 ? pm.rows : nfull;
     const int h = blockIdx.y, b = blockIdx.z;
     const int c16 = threadIdx.x & 15;
     const int rg = threadIdx.x >> 4;
@@ -119,7 +124,7 @@ __global__ void __launch_bounds__(POOL_THREADS) moba_pool_kernel(const uint16_t*
 #pragma unroll
         for (int g = 0; g < 16; ++g) s = is_max ? fmax(s, red[g][threadIdx.x]) : s + red[g][threadIdx.x];
         x = is_max ? s : s / wsum;
-        kbar[(((int64_t)b * Hkv + h) * nfull + j) * MOBA_D + threadIdx.x] = x;
+        kbar[(((int64_t)b * Hkv + h) * krows + j) * MOBA_D + threadIdx.x] = x;
     }
     if (aux.planes == nullptr) return;
     // centre and residual planes (threads 0..127 own one feature each)

@@ -20,6 +20,7 @@
 #include "k_attn_common.cuh"
 #include "k_attn_simt.cuh"
 #include "k_attn_tc.cuh"
+#include "k_decode.cuh"
 #include "k_gate.cuh"
 #include "k_gate_tc.cuh"
 #include "k_invert.cuh"
@@ -660,6 +661,162 @@ int moba_set_gate_impl(int impl) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- decode step
+namespace {
+
+struct DecodePlan {
+    int64_t c, umax, nch, nfull_needed;
+    size_t off_count, off_list, off_mask, off_part, total;
+};
+
+int make_decode_plan(int B, int Hq, int Hkv, int64_t L, int d, int bs, int topk, int full, DecodePlan* dp) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || bs < 1 || topk < 1 || d != MOBA_D || Hq % Hkv != 0) return MOBA_ERR_SHAPE;
+    if (topk > MOBA_MAX_TOPK || Hq / Hkv > DEC_MAX_G || (full != 0 && full != 1)) return MOBA_ERR_SHAPE;
+    if (B > 65535 || Hkv > 65535 || L >= ((int64_t)1 << 31) || cdiv(L, bs) > MOBA_MAX_BLOCKS) return MOBA_ERR_SHAPE;
+    const int G = Hq / Hkv;
+    dp->c = (L - 1) / bs;
+    dp->nfull_needed = dp->c;  // summaries of the earlier blocks 0 .. c - 1
+    const int64_t kp = topk - 1;
+    const int64_t past = full ? dp->c : (dp->c < (int64_t)G * kp ? dp->c : (int64_t)G * kp);
+    dp->umax = past + 1;
+    dp->nch = cdiv(bs, DEC_CHUNK);
+    const int64_t units = (int64_t)B * Hkv;
+    size_t o = 0;
+    dp->off_count = o;
+    o = align256(o + sizeof(int32_t) * (size_t)units);
+    dp->off_list = o;
+    o = align256(o + sizeof(int32_t) * (size_t)(units * dp->umax));
+    dp->off_mask = o;
+    o = align256(o + sizeof(uint32_t) * (size_t)(units * dp->umax));
+    dp->off_part = o;
+    o = align256(o + sizeof(float) * (size_t)(units * dp->umax * dp->nch * G * DEC_PART));
+    dp->total = o;
+    return MOBA_OK;
+}
+
+template <int G>
+void launch_decode_attend(const DecodeParams& p, cudaStream_t st) {
+    dim3 grid((unsigned)(p.umax * p.nch), p.Hkv, p.B);
+    moba_decode_attend_kernel<G><<<grid, DEC_THREADS, 0, st>>>(p);
+}
+
+}  // namespace
+
+extern "C" int moba_decode_workspace_size(int B, int Hq, int Hkv, int64_t L, int d, int block_size, int topk,
+                                          int full_attention, size_t* bytes) {
+    if (!bytes) return MOBA_ERR_NULL;
+    DecodePlan dp;
+    const int rc = make_decode_plan(B, Hq, Hkv, L, d, block_size, topk, full_attention, &dp);
+    if (rc) return rc;
+    *bytes = dp.total;
+    return MOBA_OK;
+}
+
+extern "C" int moba_pool_cache(const void* k, double* kbar, int B, int Hkv, int64_t L, int64_t Lmax, int d,
+                               int block_size, int64_t kbar_rows, int64_t first_block, const moba_options* options,
+                               moba_stream_t stream) {
+    if (B < 1 || Hkv < 1 || L < 0 || Lmax < L || d != MOBA_D || block_size < 1 || first_block < 0) return MOBA_ERR_SHAPE;
+    if (B > 65535 || Hkv > 65535 || Lmax >= ((int64_t)1 << 31) || (int64_t)B * Lmax >= ((int64_t)1 << 31))
+        return MOBA_ERR_SHAPE;
+    const int64_t nfull = L / block_size;
+    if (kbar_rows < nfull) return MOBA_ERR_SHAPE;
+    int rc = check_ptrs({k, (const void*)kbar});
+    if (rc) return rc;
+    PoolMode pm;
+    bool full = false;
+    if ((rc = parse_options(options, &pm, &full))) return rc;
+    if ((rc = check_device())) return rc;
+    if (first_block >= nfull) return MOBA_OK;  // nothing newly full
+    pm.j0 = first_block;
+    pm.rows = kbar_rows;
+    dim3 grid((unsigned)(nfull - first_block), Hkv, B);
+    moba_pool_kernel<<<grid, POOL_THREADS, 0, (cudaStream_t)stream>>>((const uint16_t*)k, kbar, Lmax, Hkv, block_size,
+                                                                        nfull, PoolAux{nullptr, nullptr, nullptr}, pm);
+    count_launch();
+    return launch_ok();
+}
+
+extern "C" int moba_decode(const void* q, const void* k, const void* v, const double* kbar, int64_t kbar_rows,
+                           void* out, float* lse, int32_t* idx, int B, int Hq, int Hkv, int64_t L, int64_t Lmax, int d,
+                           int block_size, int topk, int full_attention, void* workspace, size_t workspace_bytes,
+                           moba_stream_t stream) {
+    DecodePlan dp;
+    int rc = make_decode_plan(B, Hq, Hkv, L, d, block_size, topk, full_attention, &dp);
+    if (rc) return rc;
+    if (Lmax < L || (int64_t)B * Lmax >= ((int64_t)1 << 31)) return MOBA_ERR_SHAPE;
+    if (!full_attention && kbar_rows < dp.nfull_needed) return MOBA_ERR_SHAPE;
+    if ((rc = check_ptrs({q, k, v, out, (const void*)lse}))) return rc;
+    if (!full_attention && dp.c > 0 && !kbar) return MOBA_ERR_NULL;
+    if ((kbar && !aligned16(kbar)) || (idx && !aligned16(idx))) return MOBA_ERR_ALIGN;
+    if ((rc = check_device())) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    bool own = false;
+    char* ws = (char*)workspace;
+    if (!ws) {
+        if (cudaMallocAsync((void**)&ws, dp.total, st) != cudaSuccess) {
+            cudaGetLastError();
+            return MOBA_ERR_OOM;
+        }
+        own = true;
+    } else if (workspace_bytes < dp.total || ((uintptr_t)ws & 255)) {
+        return MOBA_ERR_WORKSPACE;
+    }
+    DecodeParams p;
+    p.q = (const uint16_t*)q;
+    p.k = (const uint16_t*)k;
+    p.v = (const uint16_t*)v;
+    p.kbar = kbar;
+    p.kbar_rows = kbar_rows;
+    p.L = L;
+    p.Lmax = Lmax;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.bs = block_size;
+    p.topk = topk;
+    p.c = dp.c;
+    p.umax = dp.umax;
+    p.nch = dp.nch;
+    p.full = full_attention;
+    p.ucount = (int32_t*)(ws + dp.off_count);
+    p.ulist = (int32_t*)(ws + dp.off_list);
+    p.umask = (uint32_t*)(ws + dp.off_mask);
+    p.part = (float*)(ws + dp.off_part);
+    p.idx_out = full_attention ? nullptr : idx;
+    p.out = (uint16_t*)out;
+    p.lse = lse;
+    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
+    do {
+        const size_t smem_sel = sizeof(double) * (size_t)(dp.c > 0 ? dp.c : 1) +
+                                sizeof(int32_t) * (size_t)p.G * (size_t)(topk > 1 ? topk - 1 : 1);
+        cudaError_t e = cudaFuncSetAttribute(moba_decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem_sel);
+        if (e != cudaSuccess) {
+            rc = cuda_fail(e);
+            break;
+        }
+        moba_decode_select_kernel<<<dim3(Hkv, B), DEC_THREADS, full_attention ? 0 : smem_sel, st>>>(p);
+        count_launch();
+        if ((rc = launch_ok())) break;
+        switch (p.G) {
+            case 1: launch_decode_attend<1>(p, st); break;
+            case 2: launch_decode_attend<2>(p, st); break;
+            case 3: launch_decode_attend<3>(p, st); break;
+            case 4: launch_decode_attend<4>(p, st); break;
+            case 5: case 6: case 7: case 8: launch_decode_attend<8>(p, st); break;
+            default: launch_decode_attend<16>(p, st); break;  // 9 .. 16 (make_decode_plan caps G)
+        }
+        count_launch();
+        if ((rc = launch_ok())) break;
+        moba_decode_merge_kernel<<<dim3(Hq, B), DEC_THREADS, 0, st>>>(p);
+        count_launch();
+        rc = launch_ok();
+    } while (0);
+    if (own) cudaFreeAsync(ws, st);
+    return rc;
+}
 
 // ---------------------------------------------------------------- allocation-free gate
 // Some callers cannot allocate device memory while they run: serving engines

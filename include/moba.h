@@ -210,6 +210,46 @@ int moba_stage_timing(int enable);
 int moba_stage_times(float* ms, int n, int* calls);
 
 /*
+ * ---------------------------------------------------------------- decode step
+ * One new query per sequence against its KV cache, with the prefill's gate: the query is the
+ * token at position L - 1, scores the earlier full blocks j < c = floor((L - 1) / block_size) as
+ * <q, Kbar_j>, keeps its own block c and the topk - 1 best earlier ones, and attends their keys
+ * (the own block up to L - 1). Definition: "MoBA project hub" page, Steps 2-3, and "MoBA
+ * tech-report summary" page, section 2, at the last row of the prefill. full_attention = 1 keeps
+ * every block (a full-attention layer of a hybrid model; "KIMI MoBA" blog, section 3,
+ * hybrid_layers: the pages decode with full attention).
+ *
+ * Layouts: q, out bf16 [B, Hq, d]; k, v bf16 [B, Lmax, Hkv, d] (a cache with room for Lmax tokens
+ * per sequence, the first L filled; every sequence of the batch has length L); lse fp32 [B, Hq];
+ * kbar fp64 [B, Hkv, kbar_rows, d], the block summaries written by moba_pool_cache; idx (optional,
+ * may be NULL; not written with full_attention) int32 [B, Hq, topk], the kept blocks ascending,
+ * own block last, -1 padded. Supported: Hq / Hkv <= 16, plus the limits above.
+ */
+
+/* Bytes of device workspace moba_decode needs. No device work. */
+int moba_decode_workspace_size(int B, int Hq, int Hkv, int64_t L, int d, int block_size, int topk,
+                               int full_attention, size_t* bytes);
+
+/*
+ * Block summaries of a KV cache for the gate of moba_decode: pools the full blocks
+ * first_block .. floor(L / block_size) - 1 of k (bf16 [B, Lmax, Hkv, d]) into rows of kbar
+ * (fp64 [B, Hkv, kbar_rows, d], kbar_rows >= floor(L / block_size)) with the options' pooling
+ * (NULL: mean). A decoder that appends tokens pools each block once, when it becomes full.
+ */
+int moba_pool_cache(const void* k, double* kbar, int B, int Hkv, int64_t L, int64_t Lmax, int d,
+                    int block_size, int64_t kbar_rows, int64_t first_block, const moba_options* options,
+                    moba_stream_t stream);
+
+/*
+ * The decode step. kbar must hold the summaries of blocks 0 .. c - 1 (kbar_rows >= c; not read
+ * with full_attention, may then be NULL). A NULL workspace is allocated with cudaMallocAsync on
+ * `stream`; otherwise at least moba_decode_workspace_size() bytes, 256-byte aligned.
+ */
+int moba_decode(const void* q, const void* k, const void* v, const double* kbar, int64_t kbar_rows, void* out,
+                float* lse, int32_t* idx, int B, int Hq, int Hkv, int64_t L, int64_t Lmax, int d, int block_size,
+                int topk, int full_attention, void* workspace, size_t workspace_bytes, moba_stream_t stream);
+
+/*
  * moba_gate without any device allocation, for callers that cannot allocate
  * while they run (serving engines that pre-plan every byte of HBM for their KV
  * cache, embedders with a fixed memory budget). The MoBA pages have no
