@@ -155,6 +155,30 @@ def forward(q, k, v, block_size: int, topk: int, rows: np.ndarray | None = None,
     return {"rows": rows, "sel": sel, "s_last": s_last, "s_next": s_next, "out": out, "lse": lse}
 
 
+def forward_varlen(q, k, v, cu_seqlens, block_size: int, topk: int, pooling: str = "mean", weights=None):
+    """Packed sequences: q [total, Hq, d], k, v [total, Hkv, d], sequence s holding tokens
+    cu_seqlens[s] .. cu_seqlens[s+1] - 1. Reading: each sequence is its own context (its blocks start
+    at its first token; no query reads another sequence's keys), so the method is applied to each
+    sequence on its own. Returns sel [Hq, total, topk], out [total, Hq, d], lse [Hq, total]."""
+    _check_bf16(q.unsqueeze(0), k.unsqueeze(0), v.unsqueeze(0))
+    total, Hq, d = q.shape
+    sel = np.full((Hq, total, topk), -1, dtype=np.int32)
+    out = np.zeros((total, Hq, d))
+    lse = np.zeros((Hq, total))
+    cu = [int(x) for x in cu_seqlens]
+    for s in range(len(cu) - 1):
+        a, b = cu[s], cu[s + 1]
+        if b <= a:
+            continue
+        r = forward(q[a:b].unsqueeze(0).contiguous(), k[a:b].unsqueeze(0).contiguous(),
+                    v[a:b].unsqueeze(0).contiguous(), block_size, topk, pooling=pooling, weights=weights)
+        rows = r["rows"]
+        sel[rows[:, 1], a + rows[:, 2]] = r["sel"]
+        out[a + rows[:, 2], rows[:, 1]] = r["out"]
+        lse[rows[:, 1], a + rows[:, 2]] = r["lse"]
+    return {"sel": sel, "out": out, "lse": lse}
+
+
 def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_size: int, topk: int, length: int,
            pooling: str = "mean", weights=None, full_attention: bool = False):
     """One decode step: the query q [B, Hq, d] is the token at position length - 1 of each sequence,
