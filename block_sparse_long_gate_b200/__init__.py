@@ -40,6 +40,7 @@ EXPORTED = [
     "moba_set_attention_impl", "moba_set_gate_impl", "moba_stage_timing", "moba_stage_times",
     "moba_launch_count", "moba_gate_noalloc", "moba_last_error_string", "moba_selftest_wait_timeout",
     "moba_forward_ex", "moba_gate_ex", "moba_decode_workspace_size", "moba_pool_cache", "moba_decode",
+    "moba_varlen_workspace_size", "moba_forward_varlen", "moba_gate_varlen",
 ]
 STAGES = ("pool", "gate", "invert", "attention", "merge")
 
@@ -118,6 +119,15 @@ def lib():
             L.moba_decode.restype = _I
             L.moba_decode.argtypes = [_P, _P, _P, _P, _L, _P, _P, _P, _I, _I, _I, _L, _L, _I, _I, _I, _I, _P,
                                       ctypes.c_size_t, _P]
+            _LP = ctypes.POINTER(ctypes.c_int64)
+            L.moba_varlen_workspace_size.restype = _I
+            L.moba_varlen_workspace_size.argtypes = [_LP, _I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]
+            L.moba_forward_varlen.restype = _I
+            L.moba_forward_varlen.argtypes = [_P, _P, _P, _P, _P, _LP, _I, _I, _I, _I, _I, _I, ctypes.POINTER(Options),
+                                              _P, ctypes.c_size_t, _P]
+            L.moba_gate_varlen.restype = _I
+            L.moba_gate_varlen.argtypes = [_P, _P, _P, _LP, _I, _I, _I, _I, _I, _I, ctypes.POINTER(Options), _P,
+                                           ctypes.c_size_t, _P]
             L.moba_gate_noalloc.restype = _I
             L.moba_gate_noalloc.argtypes = [_P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P]
             _lib = L
@@ -249,6 +259,62 @@ def forward_selected(q, k, v, idx, block_size: int, topk: int, out=None, lse=Non
                                           N, d, block_size, topk, _ptr(workspace), workspace.numel(),
                                           _stream(stream)), "moba_forward_selected_ws")
     return out, lse
+
+
+def _cu_array(cu_seqlens):
+    vals = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    return (ctypes.c_int64 * len(vals))(*vals), len(vals) - 1
+
+
+def varlen_workspace_size(cu_seqlens, Hq, Hkv, d, block_size, topk) -> int:
+    arr, nseq = _cu_array(cu_seqlens)
+    n = ctypes.c_size_t(0)
+    _check(lib().moba_varlen_workspace_size(arr, nseq, Hq, Hkv, d, block_size, topk, ctypes.byref(n)),
+           "moba_varlen_workspace_size")
+    return int(n.value)
+
+
+def _check_packed(q, k, v=None):
+    for t in [q, k] + ([v] if v is not None else []):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+        if t.dim() != 3:
+            raise ValueError("packed q, k, v have the layout [total, H, d]")
+    return q.shape[0], q.shape[1], k.shape[1], q.shape[2]
+
+
+def forward_varlen(q, k, v, cu_seqlens, block_size: int, topk: int, out=None, lse=None, workspace=None,
+                   stream=None, pooling: str = "mean", pool_weights=None, full_attention: bool = False):
+    """Packed sequences (q [total, Hq, d], k, v [total, Hkv, d], host cu_seqlens). Returns
+    (out [total, Hq, d], lse [Hq, total])."""
+    total, Hq, Hkv, d = _check_packed(q, k, v)
+    arr, nseq = _cu_array(cu_seqlens)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((Hq, total), dtype=torch.float32, device=q.device) if lse is None else lse
+    if workspace is None:
+        workspace = torch.empty(varlen_workspace_size(cu_seqlens, Hq, Hkv, d, block_size, topk), dtype=torch.uint8,
+                                device=q.device)
+    opt = options(pooling, pool_weights, full_attention)
+    _check(lib().moba_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), arr, nseq, Hq, Hkv, d,
+                                     block_size, topk, ctypes.byref(opt), _ptr(workspace), workspace.numel(),
+                                     _stream(stream)), "moba_forward_varlen")
+    return out, lse
+
+
+def gate_varlen(q, k, cu_seqlens, block_size: int, topk: int, idx=None, workspace=None, stream=None,
+                pooling: str = "mean", pool_weights=None):
+    """Selected blocks of every packed token: int32 [Hq, total, topk]."""
+    total, Hq, Hkv, d = _check_packed(q, k)
+    arr, nseq = _cu_array(cu_seqlens)
+    idx = torch.empty((Hq, total, topk), dtype=torch.int32, device=q.device) if idx is None else idx
+    if workspace is None:
+        workspace = torch.empty(varlen_workspace_size(cu_seqlens, Hq, Hkv, d, block_size, topk), dtype=torch.uint8,
+                                device=q.device)
+    opt = options(pooling, pool_weights)
+    _check(lib().moba_gate_varlen(_ptr(q), _ptr(k), _ptr(idx), arr, nseq, Hq, Hkv, d, block_size, topk,
+                                  ctypes.byref(opt), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "moba_gate_varlen")
+    return idx
 
 
 def decode_workspace_size(B, Hq, Hkv, L, d, block_size, topk, full_attention=False) -> int:

@@ -662,6 +662,172 @@ int moba_set_gate_impl(int impl) {
 
 }  // extern "C"
 
+// ---------------------------------------------------------------- packed (varlen) batches
+// Each packed sequence is its own context. Consecutive sequences of equal length are one
+// batched call of the fixed-length path (their tokens are adjacent, so [n, len, H, d] is a view of
+// the packed [total, H, d]); lse and idx, packed as [Hq, total(, topk)], are written through a
+// buffer in the workspace and one strided 2-D copy per sequence.
+namespace {
+
+struct VarRun {
+    int64_t s0, n, len, tok0;  // first sequence, sequences, their length, first token
+};
+
+int varlen_runs(const int64_t* cu, int nseq, std::vector<VarRun>* runs, int64_t* total) {
+    if (!cu) return MOBA_ERR_NULL;
+    if (nseq < 1 || cu[0] != 0) return MOBA_ERR_SHAPE;
+    runs->clear();
+    for (int s = 0; s < nseq; ++s) {
+        const int64_t len = cu[s + 1] - cu[s];
+        if (len < 0) return MOBA_ERR_SHAPE;
+        if (len == 0) continue;
+        if (!runs->empty() && runs->back().len == len && runs->back().s0 + runs->back().n == s &&
+            runs->back().n < 65535)
+            runs->back().n += 1;
+        else
+            runs->push_back(VarRun{s, 1, len, cu[s]});
+    }
+    *total = cu[nseq];
+    if (*total >= ((int64_t)1 << 31)) return MOBA_ERR_SHAPE;
+    return MOBA_OK;
+}
+
+// Workspace of the varlen entry points: the largest run's forward workspace (or gate scratch plus
+// its selection), then the largest run's lse / idx staging buffer.
+int varlen_plan(const std::vector<VarRun>& runs, int Hq, int Hkv, int d, int bs, int topk, size_t* fwd,
+                size_t* stage, size_t* total) {
+    *fwd = 0;
+    *stage = 0;
+    for (const VarRun& r : runs) {
+        Plan P;
+        const int rc = make_plan((int)r.n, Hq, Hkv, r.len, d, bs, topk, &P);
+        if (rc) return rc;
+        const size_t gate_need = P.gate_bytes;  // the gate path keeps its selection in the staging buffer
+        *fwd = *fwd > P.total ? *fwd : P.total;
+        *fwd = *fwd > gate_need ? *fwd : gate_need;
+        const size_t st_lse = sizeof(float) * (size_t)(r.n * Hq * r.len);
+        const size_t st_idx = sizeof(int32_t) * (size_t)(r.n * Hq * r.len * topk);
+        const size_t need = st_lse > st_idx ? st_lse : st_idx;
+        *stage = *stage > need ? *stage : need;
+    }
+    *total = align256(*fwd) + align256(*stage > 0 ? *stage : 1);
+    return MOBA_OK;
+}
+
+// dst[h][tok0 + b*len + t] (row pitch total) <- src[b][h][t] for every sequence b of the run
+int varlen_scatter(void* dst, const void* src, const VarRun& r, int Hq, int64_t total, size_t elem, cudaStream_t st) {
+    for (int64_t b = 0; b < r.n; ++b) {
+        const char* s = (const char*)src + (size_t)(b * Hq * r.len) * elem;
+        char* dd = (char*)dst + (size_t)(r.tok0 + b * r.len) * elem;
+        const cudaError_t e = cudaMemcpy2DAsync(dd, (size_t)total * elem, s, (size_t)r.len * elem,
+                                                (size_t)r.len * elem, (size_t)Hq, cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return MOBA_OK;
+}
+
+}  // namespace
+
+extern "C" int moba_varlen_workspace_size(const int64_t* cu_seqlens, int nseq, int Hq, int Hkv, int d, int block_size,
+                                          int topk, size_t* bytes) {
+    if (!bytes) return MOBA_ERR_NULL;
+    std::vector<VarRun> runs;
+    int64_t total = 0;
+    int rc = varlen_runs(cu_seqlens, nseq, &runs, &total);
+    if (rc) return rc;
+    size_t fwd, stage;
+    if ((rc = varlen_plan(runs, Hq, Hkv, d, block_size, topk, &fwd, &stage, bytes))) return rc;
+    return MOBA_OK;
+}
+
+extern "C" int moba_forward_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                                   const int64_t* cu_seqlens, int nseq, int Hq, int Hkv, int d, int block_size,
+                                   int topk, const moba_options* options, void* workspace, size_t workspace_bytes,
+                                   moba_stream_t stream) {
+    std::vector<VarRun> runs;
+    int64_t total = 0;
+    int rc = varlen_runs(cu_seqlens, nseq, &runs, &total);
+    if (rc) return rc;
+    size_t fwd, stage, need;
+    if ((rc = varlen_plan(runs, Hq, Hkv, d, block_size, topk, &fwd, &stage, &need))) return rc;
+    PoolMode pm;
+    bool full = false;
+    if ((rc = parse_options(options, &pm, &full))) return rc;
+    if ((rc = check_ptrs({q, k, v, out, (const void*)lse}))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    bool own = false;
+    char* ws = (char*)workspace;
+    if (!ws) {
+        if (cudaMallocAsync((void**)&ws, need, st) != cudaSuccess) {
+            cudaGetLastError();
+            return MOBA_ERR_OOM;
+        }
+        own = true;
+    } else if (workspace_bytes < need || ((uintptr_t)ws & 255)) {
+        return MOBA_ERR_WORKSPACE;
+    }
+    float* lse_stage = (float*)(ws + align256(fwd));
+    for (const VarRun& r : runs) {
+        const size_t qoff = (size_t)r.tok0 * Hq * MOBA_D, koff = (size_t)r.tok0 * Hkv * MOBA_D;
+        const uint16_t* qr = (const uint16_t*)q + qoff;
+        const uint16_t* kr = (const uint16_t*)k + koff;
+        const uint16_t* vr = (const uint16_t*)v + koff;
+        uint16_t* orr = (uint16_t*)out + qoff;
+        if (full)
+            rc = dense_impl(qr, kr, vr, orr, lse_stage, (int)r.n, Hq, Hkv, r.len, d, st);
+        else
+            rc = forward_impl(qr, kr, vr, nullptr, orr, lse_stage, (int)r.n, Hq, Hkv, r.len, d, block_size, topk, ws,
+                              fwd, st, pm);
+        if (rc) break;
+        if ((rc = varlen_scatter(lse, lse_stage, r, Hq, total, sizeof(float), st))) break;
+    }
+    if (own) cudaFreeAsync(ws, st);
+    return rc;
+}
+
+extern "C" int moba_gate_varlen(const void* q, const void* k, int32_t* idx, const int64_t* cu_seqlens, int nseq, int Hq,
+                                int Hkv, int d, int block_size, int topk, const moba_options* options, void* workspace,
+                                size_t workspace_bytes, moba_stream_t stream) {
+    std::vector<VarRun> runs;
+    int64_t total = 0;
+    int rc = varlen_runs(cu_seqlens, nseq, &runs, &total);
+    if (rc) return rc;
+    size_t fwd, stage, need;
+    if ((rc = varlen_plan(runs, Hq, Hkv, d, block_size, topk, &fwd, &stage, &need))) return rc;
+    PoolMode pm;
+    bool full = false;
+    if ((rc = parse_options(options, &pm, &full))) return rc;
+    if (full) return MOBA_ERR_SHAPE;
+    if ((rc = check_ptrs({q, k, (const void*)idx}))) return rc;
+    if ((rc = check_device())) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    bool own = false;
+    char* ws = (char*)workspace;
+    if (!ws) {
+        if (cudaMallocAsync((void**)&ws, need, st) != cudaSuccess) {
+            cudaGetLastError();
+            return MOBA_ERR_OOM;
+        }
+        own = true;
+    } else if (workspace_bytes < need || ((uintptr_t)ws & 255)) {
+        return MOBA_ERR_WORKSPACE;
+    }
+    int32_t* idx_stage = (int32_t*)(ws + align256(fwd));
+    for (const VarRun& r : runs) {
+        Plan P;
+        if ((rc = make_plan((int)r.n, Hq, Hkv, r.len, d, block_size, topk, &P))) break;
+        const GateScratch gs = gate_scratch(P, ws, use_tc_gate(P));
+        const uint16_t* qr = (const uint16_t*)q + (size_t)r.tok0 * Hq * MOBA_D;
+        const uint16_t* kr = (const uint16_t*)k + (size_t)r.tok0 * Hkv * MOBA_D;
+        if ((rc = run_pool(P, kr, gs, pm, st))) break;
+        if ((rc = run_gate(P, qr, gs, idx_stage, st))) break;
+        if ((rc = varlen_scatter(idx, idx_stage, r, Hq, total, sizeof(int32_t) * topk, st))) break;
+    }
+    if (own) cudaFreeAsync(ws, st);
+    return rc;
+}
+
 // ---------------------------------------------------------------- decode step
 namespace {
 

@@ -210,6 +210,33 @@ int moba_stage_timing(int enable);
 int moba_stage_times(float* ms, int n, int* calls);
 
 /*
+ * ---------------------------------------------------------------- packed (varlen) batches
+ * Sequences of different lengths packed back to back, as in the pages' FlashAttention pipeline
+ * ("MoBA tech-report summary" page, section 2, implementation steps 1-5, a variable-length
+ * kernel): sequence s holds tokens cu_seqlens[s] .. cu_seqlens[s+1] - 1 and is its own context
+ * (its blocks start at its first token; no query attends another sequence's keys).
+ * Layouts: q, out bf16 [total, Hq, d]; k, v bf16 [total, Hkv, d]; lse fp32 [Hq, total];
+ * idx int32 [Hq, total, topk] (as moba_gate's rows). cu_seqlens is a HOST int64 array of
+ * nseq + 1 non-decreasing offsets starting at 0 (empty sequences allowed), total =
+ * cu_seqlens[nseq] < 2^31. Consecutive sequences of equal length run as one batch; others run
+ * one after another on `stream`. A NULL workspace is allocated with cudaMallocAsync on
+ * `stream`; otherwise at least moba_varlen_workspace_size() bytes, 256-byte aligned.
+ */
+int moba_varlen_workspace_size(const int64_t* cu_seqlens, int nseq, int Hq, int Hkv, int d, int block_size,
+                               int topk, size_t* bytes);
+
+/* The causal prefill forward of every packed sequence (options as in moba_forward_ex). */
+int moba_forward_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                        const int64_t* cu_seqlens, int nseq, int Hq, int Hkv, int d, int block_size, int topk,
+                        const moba_options* options, void* workspace, size_t workspace_bytes,
+                        moba_stream_t stream);
+
+/* The gate of every packed sequence (options as in moba_gate_ex). */
+int moba_gate_varlen(const void* q, const void* k, int32_t* idx, const int64_t* cu_seqlens, int nseq, int Hq,
+                     int Hkv, int d, int block_size, int topk, const moba_options* options, void* workspace,
+                     size_t workspace_bytes, moba_stream_t stream);
+
+/*
  * ---------------------------------------------------------------- decode step
  * One new query per sequence against its KV cache, with the prefill's gate: the query is the
  * token at position L - 1, scores the earlier full blocks j < c = floor((L - 1) / block_size) as
