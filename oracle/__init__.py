@@ -47,6 +47,8 @@ def _load():
             lib.oracle_pool.argtypes = [_P, _I, _I, _I, _I, _I, _P]
             lib.oracle_pool_mode.restype = None
             lib.oracle_pool_mode.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P]
+            lib.oracle_backward.restype = _I
+            lib.oracle_backward.argtypes = [_P, _P, _P, _P] + [_I] * 7 + [_P, _P, _P, _P]
             lib.oracle_select.restype = None
             lib.oracle_select.argtypes = [_P, _P] + [_I] * 7 + [_P, _I, _P, _P, _P, _P, _I]
             lib.oracle_attend.restype = _I
@@ -153,6 +155,30 @@ def forward(q, k, v, block_size: int, topk: int, rows: np.ndarray | None = None,
     sel, s_last, s_next = select(q, kbar, Hkv, block_size, topk, rows)
     out, lse = attend(q, k, v, block_size, topk, rows, sel)
     return {"rows": rows, "sel": sel, "s_last": s_last, "s_next": s_next, "out": out, "lse": lse}
+
+
+def backward(q, k, v, dout, block_size: int, topk: int, sel=None, pooling: str = "mean", weights=None):
+    """Gradients of sum(dout * out) through the forward with its selection held fixed (the top-k
+    choice is discrete: the block summaries get no gradient). sel: int32 [B, Hq, N, topk] for every
+    row (computed by the oracle's gate when None). Returns (dq [B, N, Hq, d], dk, dv [B, N, Hkv, d])
+    as float64 numpy arrays."""
+    _check_bf16(q, k, v, dout)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if sel is None:
+        rows = all_rows(B, Hq, N)
+        s, _, _ = select(q, pool(k, block_size, pooling, weights), Hkv, block_size, topk, rows)
+        sel = s.reshape(B, Hq, N, topk)
+    sel = np.ascontiguousarray(sel, dtype=np.int32)
+    assert sel.shape == (B, Hq, N, topk)
+    dq = np.zeros((B, N, Hq, d))
+    dk = np.zeros((B, N, Hkv, d))
+    dv = np.zeros((B, N, Hkv, d))
+    bad = _load().oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), B, N, Hq, Hkv, d, block_size, topk,
+                                  _ptr(sel), _ptr(dq), _ptr(dk), _ptr(dv))
+    if bad:
+        raise ValueError(f"{bad} rows name a future block, repeat a block or lack their own block")
+    return dq, dk, dv
 
 
 def forward_varlen(q, k, v, cu_seqlens, block_size: int, topk: int, pooling: str = "mean", weights=None):

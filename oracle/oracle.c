@@ -332,3 +332,109 @@ int64_t oracle_attend_blockwise(const uint16_t* Q, const uint16_t* K, const uint
     }
     return bad;
 }
+
+/*
+ * Step 7 (the backward of steps 5-6, for training: "MoBA tech-report summary", section 3
+ * trains and continues pre-training models with MoBA). With the selection fixed (the top-k
+ * choice is discrete, so the block representatives receive no gradient; only the attention is
+ * differentiated), for the loss sum over rows of <dO_t, out_t>:
+ *   P_tu = exp(l_u - lse_t) over the row's allowed keys u, l_u = q_t.k_u / sqrt(d)
+ *   D_t  = sum_e dO_t[e] out_t[e]
+ *   dP_tu = dO_t . v_u,   dS_tu = P_tu (dP_tu - D_t)
+ *   dQ_t = sum_u dS_tu k_u / sqrt(d),  dK_u += dS_tu q_t / sqrt(d),  dV_u += P_tu dO_t
+ * with out_t and lse_t the row's own forward (recomputed here in fp64). GQA: a kv head sums the
+ * contributions of its query heads. sel: [B, Hq, N, topk] for every row. Outputs in fp64:
+ * dQ [B, N, Hq, d], dK and dV [B, N, Hkv, d] (zeroed here). Returns the number of rows whose
+ * selection was malformed (left without contributions).
+ */
+int64_t oracle_backward(const uint16_t* Q, const uint16_t* K, const uint16_t* V, const uint16_t* dO,
+                        int64_t B, int64_t N, int64_t Hq, int64_t Hkv, int64_t d, int64_t bs,
+                        int64_t topk, const int32_t* sel, double* dQ, double* dK, double* dV) {
+    int64_t G = Hq / Hkv;
+    double scale = 1.0 / sqrt((double)d);
+    int64_t bad = 0;
+    memset(dQ, 0, sizeof(double) * (size_t)(B * N * Hq * d));
+    memset(dK, 0, sizeof(double) * (size_t)(B * N * Hkv * d));
+    memset(dV, 0, sizeof(double) * (size_t)(B * N * Hkv * d));
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(+ : bad)
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t hk = 0; hk < Hkv; ++hk) {
+            /* one (b, kv head) per thread: its dK / dV rows are written by this thread only */
+            double* qv = (double*)malloc(sizeof(double) * (size_t)d);
+            double* gv = (double*)malloc(sizeof(double) * (size_t)d);
+            double* ov = (double*)malloc(sizeof(double) * (size_t)d);
+            double* logit = (double*)malloc(sizeof(double) * (size_t)(topk * bs + 1));
+            int64_t* key = (int64_t*)malloc(sizeof(int64_t) * (size_t)(topk * bs + 1));
+            for (int64_t g = 0; g < G; ++g) {
+                int64_t hq = hk * G + g;
+                for (int64_t t = 0; t < N; ++t) {
+                    int64_t c = t / bs;
+                    const int32_t* sr = sel + ((b * Hq + hq) * N + t) * topk;
+                    int has_own = 0, ok = 1;
+                    for (int64_t i = 0; i < topk; ++i) {
+                        if (sr[i] == c) has_own = 1;
+                        if (sr[i] > c) ok = 0;
+                        for (int64_t i2 = 0; i2 < i; ++i2)
+                            if (sr[i] >= 0 && sr[i2] == sr[i]) ok = 0;
+                    }
+                    if (!ok || !has_own) {
+                        bad += 1;
+                        continue;
+                    }
+                    for (int64_t e = 0; e < d; ++e) {
+                        qv[e] = bf16_to_double(Q[((b * N + t) * Hq + hq) * d + e]);
+                        gv[e] = bf16_to_double(dO[((b * N + t) * Hq + hq) * d + e]);
+                    }
+                    int64_t n = 0;
+                    double m = -INFINITY;
+                    for (int64_t i = 0; i < topk; ++i) {
+                        int64_t lo, hi;
+                        if (block_range(sr[i], t, bs, &lo, &hi) != 1) continue;
+                        for (int64_t u = lo; u < hi; ++u) {
+                            const uint16_t* kr = K + ((b * N + u) * Hkv + hk) * d;
+                            double s = 0.0;
+                            for (int64_t e = 0; e < d; ++e) s += qv[e] * bf16_to_double(kr[e]);
+                            logit[n] = s * scale;
+                            key[n] = u;
+                            if (logit[n] > m) m = logit[n];
+                            ++n;
+                        }
+                    }
+                    double z = 0.0;
+                    for (int64_t i = 0; i < n; ++i) z += exp(logit[i] - m);
+                    double L = m + log(z);
+                    /* the row's output and D */
+                    for (int64_t e = 0; e < d; ++e) ov[e] = 0.0;
+                    for (int64_t i = 0; i < n; ++i) {
+                        double p = exp(logit[i] - L);
+                        const uint16_t* vr = V + ((b * N + key[i]) * Hkv + hk) * d;
+                        for (int64_t e = 0; e < d; ++e) ov[e] += p * bf16_to_double(vr[e]);
+                    }
+                    double D = 0.0;
+                    for (int64_t e = 0; e < d; ++e) D += gv[e] * ov[e];
+                    double* dq = dQ + ((b * N + t) * Hq + hq) * d;
+                    for (int64_t i = 0; i < n; ++i) {
+                        double p = exp(logit[i] - L);
+                        const uint16_t* kr = K + ((b * N + key[i]) * Hkv + hk) * d;
+                        const uint16_t* vr = V + ((b * N + key[i]) * Hkv + hk) * d;
+                        double dp = 0.0;
+                        for (int64_t e = 0; e < d; ++e) dp += gv[e] * bf16_to_double(vr[e]);
+                        double ds = p * (dp - D);
+                        double* dk = dK + ((b * N + key[i]) * Hkv + hk) * d;
+                        double* dv = dV + ((b * N + key[i]) * Hkv + hk) * d;
+                        for (int64_t e = 0; e < d; ++e) {
+                            dq[e] += ds * bf16_to_double(kr[e]) * scale;
+                            dk[e] += ds * qv[e] * scale;
+                            dv[e] += p * gv[e];
+                        }
+                    }
+                }
+            }
+            free(qv);
+            free(gv);
+            free(ov);
+            free(logit);
+            free(key);
+        }
+    return bad;
+}
