@@ -40,7 +40,8 @@ EXPORTED = [
     "moba_set_attention_impl", "moba_set_gate_impl", "moba_stage_timing", "moba_stage_times",
     "moba_launch_count", "moba_gate_noalloc", "moba_last_error_string", "moba_selftest_wait_timeout",
     "moba_forward_ex", "moba_gate_ex", "moba_decode_workspace_size", "moba_pool_cache", "moba_decode",
-    "moba_varlen_workspace_size", "moba_forward_varlen", "moba_gate_varlen",
+    "moba_varlen_workspace_size", "moba_forward_varlen", "moba_gate_varlen", "moba_backward_workspace_size",
+    "moba_backward",
 ]
 STAGES = ("pool", "gate", "invert", "attention", "merge")
 
@@ -128,6 +129,11 @@ def lib():
             L.moba_gate_varlen.restype = _I
             L.moba_gate_varlen.argtypes = [_P, _P, _P, _LP, _I, _I, _I, _I, _I, _I, ctypes.POINTER(Options), _P,
                                            ctypes.c_size_t, _P]
+            L.moba_backward_workspace_size.restype = _I
+            L.moba_backward_workspace_size.argtypes = [_I, _I, _I, _L, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)]
+            L.moba_backward.restype = _I
+            L.moba_backward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P,
+                                        ctypes.c_size_t, _P]
             L.moba_gate_noalloc.restype = _I
             L.moba_gate_noalloc.argtypes = [_P, _P, _P, _I, _I, _I, _L, _I, _I, _I, _P]
             _lib = L
@@ -361,6 +367,33 @@ def decode(q, k, v, kbar, block_size: int, topk: int, length: int, full_attentio
                              Hkv, length, Lmax, d, block_size, topk, 1 if full_attention else 0, _ptr(workspace),
                              workspace.numel(), _stream(stream)), "moba_decode")
     return out, lse, idx
+
+
+def backward_workspace_size(B, Hq, Hkv, N, d, block_size, topk) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moba_backward_workspace_size(B, Hq, Hkv, N, d, block_size, topk, ctypes.byref(n)),
+           "moba_backward_workspace_size")
+    return int(n.value)
+
+
+def backward(q, k, v, out, lse, dout, block_size: int, topk: int, idx=None, dq=None, dk=None, dv=None,
+             workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of sum(dout * out) through the forward with its selection held fixed.
+    out, lse: the forward's results; idx: the forward's selection (None: the gate runs again)."""
+    B, N, Hq, Hkv, d = _check_qkv(q, k, v)
+    for t in (out, dout):
+        if t.shape != q.shape or t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("out and dout must be contiguous bf16 CUDA tensors shaped like q")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(backward_workspace_size(B, Hq, Hkv, N, d, block_size, topk), dtype=torch.uint8,
+                                device=q.device)
+    _check(lib().moba_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(idx), _ptr(dq),
+                               _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, block_size, topk, _ptr(workspace),
+                               workspace.numel(), _stream(stream)), "moba_backward")
+    return dq, dk, dv
 
 
 def dense_causal(q, k, v, out=None, lse=None, stream=None):

@@ -20,6 +20,7 @@
 #include "k_attn_common.cuh"
 #include "k_attn_simt.cuh"
 #include "k_attn_tc.cuh"
+#include "k_backward.cuh"
 #include "k_decode.cuh"
 #include "k_gate.cuh"
 #include "k_gate_tc.cuh"
@@ -661,6 +662,139 @@ int moba_set_gate_impl(int impl) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- backward
+namespace {
+
+// The forward plan's gate scratch, selection and inversion arrays, then D, the fp32 dq
+// accumulator and the work counter (the forward's partials are not needed).
+struct BwdPlan {
+    Plan P;
+    size_t off_D, off_acc, off_counter, total;
+};
+
+int make_bwd_plan(int B, int Hq, int Hkv, int64_t N, int d, int bs, int topk, BwdPlan* bp) {
+    int rc = make_plan(B, Hq, Hkv, N, d, bs, topk, &bp->P);
+    if (rc) return rc;
+    size_t o = bp->P.off_opart;  // everything before the partials
+    bp->off_D = o;
+    o = align256(o + sizeof(float) * (size_t)B * Hq * N);
+    bp->off_acc = o;
+    o = align256(o + sizeof(float) * (size_t)B * N * Hq * MOBA_D);
+    bp->off_counter = o;
+    o = align256(o + sizeof(int));
+    bp->total = o;
+    return MOBA_OK;
+}
+
+}  // namespace
+
+extern "C" int moba_backward_workspace_size(int B, int Hq, int Hkv, int64_t N, int d, int block_size, int topk,
+                                            size_t* bytes) {
+    if (!bytes) return MOBA_ERR_NULL;
+    BwdPlan bp;
+    const int rc = make_bwd_plan(B, Hq, Hkv, N, d, block_size, topk, &bp);
+    if (rc) return rc;
+    *bytes = bp.total;
+    return MOBA_OK;
+}
+
+extern "C" int moba_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                             const void* dout, const int32_t* idx, void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                             int64_t N, int d, int block_size, int topk, void* workspace, size_t workspace_bytes,
+                             moba_stream_t stream) {
+    BwdPlan bp;
+    int rc = make_bwd_plan(B, Hq, Hkv, N, d, block_size, topk, &bp);
+    if (rc) return rc;
+    const Plan& P = bp.P;
+    if ((rc = check_ptrs({q, k, v, out, (const void*)lse, dout, dq, dk, dv}))) return rc;
+    if (idx && !aligned16(idx)) return MOBA_ERR_ALIGN;
+    if ((rc = check_device())) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    bool own = false;
+    char* ws = (char*)workspace;
+    if (!ws) {
+        if (cudaMallocAsync((void**)&ws, bp.total, st) != cudaSuccess) {
+            cudaGetLastError();
+            return MOBA_ERR_OOM;
+        }
+        own = true;
+    } else if (workspace_bytes < bp.total || ((uintptr_t)ws & 255)) {
+        return MOBA_ERR_WORKSPACE;
+    }
+    do {
+        // the selection: the caller's (checked row by row by the inversion), or the gate's again
+        const int32_t* sel = idx;
+        if (!sel) {
+            int32_t* widx = (int32_t*)(ws + P.off_idx);
+            const GateScratch gs = gate_scratch(P, ws, use_tc_gate(P));
+            if ((rc = run_pool(P, k, gs, PoolMode{0, nullptr}, st))) break;
+            if ((rc = run_gate(P, q, gs, widx, st))) break;
+            sel = widx;
+        }
+        if ((rc = run_invert(P, sel, ws, st))) break;
+        float* D = (float*)(ws + bp.off_D);
+        float* acc = (float*)(ws + bp.off_acc);
+        int* counter = (int*)(ws + bp.off_counter);
+        const int64_t nrows = (int64_t)B * Hq * N;
+        moba_bwd_prep_kernel<<<(unsigned)cdiv(nrows * 16, 256), 256, 0, st>>>((const uint16_t*)out,
+                                                                              (const uint16_t*)dout, D, N, Hq, nrows);
+        count_launch();
+        if ((rc = launch_ok())) break;
+        cudaError_t e = cudaMemsetAsync(acc, 0, sizeof(float) * (size_t)B * N * Hq * MOBA_D, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(counter, 0, sizeof(int), st);
+        if (e != cudaSuccess) {
+            rc = cuda_fail(e);
+            break;
+        }
+        BwdParams bpar;
+        bpar.q = (const uint16_t*)q;
+        bpar.dout = (const uint16_t*)dout;
+        bpar.lse = lse;
+        bpar.Dvec = D;
+        bpar.dk = (uint16_t*)dk;
+        bpar.dv = (uint16_t*)dv;
+        bpar.dq_acc = acc;
+        bpar.entries = (const uint64_t*)(ws + P.off_entries);
+        bpar.segoff = (const int64_t*)(ws + P.off_segoff);
+        bpar.counter = counter;
+        bpar.N = N;
+        bpar.nblk = P.nblk;
+        bpar.nch = P.nch;
+        bpar.mb = P.mb;
+        bpar.items = P.L * P.mb;
+        bpar.B = B;
+        bpar.Hq = Hq;
+        bpar.Hkv = Hkv;
+        bpar.G = P.G;
+        bpar.bs = block_size;
+        bpar.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
+        bpar.scale = (float)(1.0 / sqrt((double)d));
+        TcMaps maps;
+        if (!moba_make_kv_map(&maps.k, k, (int64_t)B * N, Hkv) || !moba_make_kv_map(&maps.v, v, (int64_t)B * N, Hkv)) {
+            rc = MOBA_ERR_CUDA;
+            break;
+        }
+        int dev = 0, nsm = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(moba_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      BWD_SMEM_BYTES)) != cudaSuccess) {
+            rc = cuda_fail(e);
+            break;
+        }
+        const int64_t grid = bpar.items < nsm ? bpar.items : nsm;
+        moba_bwd_kernel<<<(unsigned)grid, BWD_THREADS, BWD_SMEM_BYTES, st>>>(bpar, maps);
+        count_launch();
+        if ((rc = launch_ok())) break;
+        const int64_t n4 = (int64_t)B * N * Hq * MOBA_D / 4;
+        moba_bwd_dq_kernel<<<(unsigned)cdiv(n4, 256), 256, 0, st>>>(acc, (uint16_t*)dq, bpar.scale, n4);
+        count_launch();
+        rc = launch_ok();
+    } while (0);
+    if (own) cudaFreeAsync(ws, st);
+    return rc;
+}
 
 // ---------------------------------------------------------------- packed (varlen) batches
 // Each packed sequence is its own context. Consecutive sequences of equal length are one

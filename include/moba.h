@@ -210,6 +210,29 @@ int moba_stage_timing(int enable);
 int moba_stage_times(float* ms, int n, int* calls);
 
 /*
+ * ---------------------------------------------------------------- backward
+ * Gradients of sum(dout * out) for the causal prefill forward, with its selection held fixed:
+ * the top-k choice is discrete, so gradients flow only through the attention over the kept keys
+ * and the block summaries receive none ("MoBA tech-report summary" page, section 3, trains and
+ * continues pre-training models with MoBA; the attention is softmax(q k^T / sqrt(d)) v as in the
+ * "NSA vs MoBA" blog, section 1).
+ *   dq = sum_u dS_tu k_u / sqrt(d), dk = sum_t dS_tu q_t / sqrt(d), dv = sum_t P_tu dout_t,
+ *   P_tu = exp(q_t.k_u / sqrt(d) - lse_t), dS_tu = P_tu (dout_t.v_u - <dout_t, out_t>).
+ * Inputs: q, k, v, out (the forward's output) and dout in the forward's layouts, lse fp32
+ * [B, Hq, N] (the forward's); idx: the forward's selection (int32 [B, Hq, N, topk], as moba_gate
+ * writes it) or NULL to run the gate again (same result). Outputs dq [B, N, Hq, d], dk, dv
+ * [B, N, Hkv, d], bf16. A NULL workspace is allocated with cudaMallocAsync on `stream`;
+ * otherwise at least moba_backward_workspace_size() bytes, 256-byte aligned.
+ */
+int moba_backward_workspace_size(int B, int Hq, int Hkv, int64_t N, int d, int block_size, int topk,
+                                 size_t* bytes);
+
+int moba_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                  const void* dout, const int32_t* idx, void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                  int64_t N, int d, int block_size, int topk, void* workspace, size_t workspace_bytes,
+                  moba_stream_t stream);
+
+/*
  * ---------------------------------------------------------------- packed (varlen) batches
  * Sequences of different lengths packed back to back, as in the pages' FlashAttention pipeline
  * ("MoBA tech-report summary" page, section 2, implementation steps 1-5, a variable-length
