@@ -84,8 +84,9 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-sdpa", action="store_true", help="skip torch's dense attention in the dense arm")
-    p.add_argument("--mode", choices=("prefill", "decode"), default="prefill",
-                   help="decode: one new query per sequence against a KV cache of the workload's length")
+    p.add_argument("--mode", choices=("prefill", "decode", "backward"), default="prefill",
+                   help="decode: one new query per sequence against a KV cache of the workload's length; "
+                        "backward: dq, dk, dv of the workload's forward")
     p.add_argument("--pooling", choices=("mean", "max", "weighted"), default="mean",
                    help="the gate's block summary (weighted: weights rising linearly from 0.5 to 1.5 across a block)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -731,12 +732,77 @@ def run_decode(args):
     return 0
 
 
+def run_backward(args):
+    """The backward of the workload's forward (dq, dk, dv through its selection), timed on its own:
+    useful work = 2.5 x the forward's useful FLOPs (five products per attended pair instead of two)."""
+    import torch
+
+    from block_sparse_long_gate_b200.build import build_library
+    build_library()
+    import block_sparse_long_gate_b200 as moba
+    from block_sparse_long_gate_b200 import flops as fx
+    import synth
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--mode backward runs on one GPU")
+    dev = torch.device("cuda", 0)
+    w = workload(args.seq_len, args.hq, args.hkv, args.config)
+    B, N, Hq, Hkv, d, bs, topk = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"], w["block_size"], w["topk"]
+    q_h, k_h, v_h = host_inputs(w, w["seed"], pin=True)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    g = synth.normal(w["seed"] + 7, synth.V_ID, (B, N, Hq, d)).to(dev)
+    out, lse = moba.forward(q, k, v, bs, topk)
+    idx = moba.gate(q, k, bs, topk)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(moba.backward_workspace_size(B, Hq, Hkv, N, d, bs, topk), dtype=torch.uint8, device=dev)
+
+    def step():
+        moba.backward(q, k, v, out, lse, g, bs, topk, idx=idx, dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else "0"
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0 = moba.launch_count()
+    with ClockSampler(gpu_id) as clk:
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(args.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    status = moba.sync_status()
+    fl = 2.5 * fx.useful_flops(B, Hq, N, d, bs, topk)
+    value = fl / (ms * 1e-3) / 1e12
+    peaks, peak_src = read_peaks()
+    sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    line = {
+        "metric": "MoBA backward useful TFLOP/s (dq, dk, dv)", "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "backward of " + workload_name(w), "global_batch": B, "seq_len": N,
+                   "parallelism": "single GPU", "l2": "inputs far exceed the 126 MB L2"},
+        "roofline": {"kernel": "moba_bwd_kernel and its helpers (whole backward)", "bound": "tensor",
+                     "achieved": value, "peak": sust, "unit": "TFLOP/s", "frac": value / sust, "traffic": None,
+                     "peak_source": f"bf16_tflops_sustained, {peak_src}"},
+        "gpu_launches": (moba.launch_count() - l0) // max(args.steps, 1), "clocks": clk.summary(),
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
     if args.mode == "decode":
         return run_decode(args)
+    if args.mode == "backward":
+        return run_backward(args)
     return run_moba(args)
 
 
