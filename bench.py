@@ -368,8 +368,8 @@ def time_sdpa(q, k, v, stream) -> dict:
 
     def attempt(kk, vv, gqa):
         with sdpa_kernel(backends):
-            F.scaled_dot_product_attention(qt[:, :, :4096], kk[:, :, :4096], vv[:, :, :4096], is_causal=True,
-                                           enable_gqa=gqa)
+            # warm up at the timed shape: a backend may build its plan for a new shape on the first call
+            F.scaled_dot_product_attention(qt, kk, vv, is_causal=True, enable_gqa=gqa)
             torch.cuda.synchronize()
             e0.record(stream)
             o = F.scaled_dot_product_attention(qt, kk, vv, is_causal=True, enable_gqa=gqa)
