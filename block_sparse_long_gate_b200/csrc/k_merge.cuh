@@ -36,7 +36,7 @@ __device__ __forceinline__ void fma8(float (&a)[8], float w, const uint4& x) {
 // latency. The slot count comes from the row's own block when the selection was
 // made by the library's gate (well formed by construction); an injected
 // selection (VALIDATE) is read and checked first.
-template <bool VALIDATE>
+template <bool VALIDATE, int NB>
 __device__ __forceinline__ void merge_row(const int32_t* __restrict__ idx, const uint16_t* __restrict__ opart,
                                           const float* __restrict__ lpart, uint16_t* out, float* lse, int64_t N,
                                           int Hq, int bs, int topk, int64_t row) {
@@ -73,9 +73,9 @@ __device__ __forceinline__ void merge_row(const int32_t* __restrict__ idx, const
         const int s = lane + 16 * r;
         lsl[r] = s < p ? lrow[s] : -INFINITY;
     }
-    uint4 x[MERGE_BATCH];
+    uint4 x[NB];
 #pragma unroll
-    for (int u = 0; u < MERGE_BATCH; ++u)
+    for (int u = 0; u < NB; ++u)
         if (u < p) x[u] = *reinterpret_cast<const uint4*>(prow + (int64_t)u * MOBA_D);
     // weights
     float m = fmaxf(fmaxf(ld, lsl[0]), fmaxf(lsl[1], fmaxf(lsl[2], lsl[3])));
@@ -104,16 +104,16 @@ __device__ __forceinline__ void merge_row(const int32_t* __restrict__ idx, const
         return __shfl_sync(hmask, wr, src_base + (s & 15));
     };
 #pragma unroll
-    for (int u = 0; u < MERGE_BATCH; ++u) {
+    for (int u = 0; u < NB; ++u) {
         const float w = weight(u);
         if (u < p) fma8(acc, w, x[u]);
     }
-    for (int s0 = MERGE_BATCH; s0 < p; s0 += MERGE_BATCH) {  // long selections: further batches
+    for (int s0 = NB; s0 < p; s0 += NB) {  // long selections: further batches
 #pragma unroll
-        for (int u = 0; u < MERGE_BATCH; ++u)
+        for (int u = 0; u < NB; ++u)
             if (s0 + u < p) x[u] = *reinterpret_cast<const uint4*>(prow + (int64_t)(s0 + u) * MOBA_D);
 #pragma unroll
-        for (int u = 0; u < MERGE_BATCH; ++u) {
+        for (int u = 0; u < NB; ++u) {
             const float w = weight(s0 + u);
             if (s0 + u < p) fma8(acc, w, x[u]);
         }
@@ -129,7 +129,9 @@ __device__ __forceinline__ void merge_row(const int32_t* __restrict__ idx, const
 
 // Persistent: each half-warp walks the rows with a stride of all half-warps of the grid
 // (short-lived blocks of a row each left the SMs partly idle between block launches).
-template <bool VALIDATE>
+// NB: slot partials loaded per batch (the smallest of 4, 8, 12, 16 that holds k - 1, so short
+// selections keep fewer registers and more rows in flight per SM).
+template <bool VALIDATE, int NB>
 __global__ void __launch_bounds__(MERGE_THREADS) moba_merge_kernel(const int32_t* __restrict__ idx,
                                                                    const uint16_t* __restrict__ opart,
                                                                    const float* __restrict__ lpart, uint16_t* out,
@@ -138,5 +140,5 @@ __global__ void __launch_bounds__(MERGE_THREADS) moba_merge_kernel(const int32_t
     const int64_t hw = (int64_t)blockIdx.x * (MERGE_THREADS / 16) + (threadIdx.x >> 4);
     const int64_t stride = (int64_t)gridDim.x * (MERGE_THREADS / 16);
     for (int64_t row = hw; row < nrows; row += stride)  // whole half-warps iterate together
-        merge_row<VALIDATE>(idx, opart, lpart, out, lse, N, Hq, bs, topk, row);
+        merge_row<VALIDATE, NB>(idx, opart, lpart, out, lse, N, Hq, bs, topk, row);
 }

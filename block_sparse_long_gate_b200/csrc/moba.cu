@@ -366,30 +366,38 @@ int run_attention(const Plan& P, const AttnParams& a, cudaStream_t st) {
     return rc;
 }
 
-template <bool VALIDATE>
+template <bool VALIDATE, int NB>
 int launch_merge(const Plan& P, const int32_t* idx, char* ws, void* out, float* lse, cudaStream_t st) {
     int64_t nrows = (int64_t)P.B * P.Hq * P.N;
     int dev = 0, nsm = 148, per_sm = 1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moba_merge_kernel<VALIDATE>, MERGE_THREADS, 0);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moba_merge_kernel<VALIDATE, NB>, MERGE_THREADS, 0);
     if (e != cudaSuccess) return cuda_fail(e);
     int64_t grid = (int64_t)nsm * (per_sm > 0 ? per_sm : 1);
     const int64_t need = cdiv(nrows, MERGE_THREADS / 16);
     if (grid > need) grid = need;
-    moba_merge_kernel<VALIDATE><<<(unsigned)grid, MERGE_THREADS, 0, st>>>(
+    moba_merge_kernel<VALIDATE, NB><<<(unsigned)grid, MERGE_THREADS, 0, st>>>(
         idx, (const uint16_t*)(ws + P.off_opart), (const float*)(ws + P.off_lpart), (uint16_t*)out, lse, P.N, P.Hq,
         P.bs, P.topk, nrows);
     count_launch();
     return launch_ok();
 }
 
+template <bool VALIDATE>
+int launch_merge_nb(const Plan& P, const int32_t* idx, char* ws, void* out, float* lse, cudaStream_t st) {
+    if (P.kp <= 4) return launch_merge<VALIDATE, 4>(P, idx, ws, out, lse, st);
+    if (P.kp <= 8) return launch_merge<VALIDATE, 8>(P, idx, ws, out, lse, st);
+    if (P.kp <= 12) return launch_merge<VALIDATE, 12>(P, idx, ws, out, lse, st);
+    return launch_merge<VALIDATE, 16>(P, idx, ws, out, lse, st);
+}
+
 // `validate`: the selection was given by the caller and is checked row by row; the gate's own
 // selections are well formed by construction.
 int run_merge(const Plan& P, const int32_t* idx, bool validate, char* ws, void* out, float* lse,
               cudaStream_t st) {
-    return validate ? launch_merge<true>(P, idx, ws, out, lse, st) : launch_merge<false>(P, idx, ws, out, lse, st);
+    return validate ? launch_merge_nb<true>(P, idx, ws, out, lse, st) : launch_merge_nb<false>(P, idx, ws, out, lse, st);
 }
 
 int forward_impl(const void* q, const void* k, const void* v, const int32_t* idx_in, void* out, float* lse,
