@@ -21,6 +21,15 @@
 
 #define MOBA_PAIR_ROWS (2 * MOBA_TILE)
 
+// A past pair as one 16-byte record, so that a role decodes an item with one load that does
+// not depend on another (and can be issued an item ahead): its first entry, its list
+// l = (b, hk, j) and its entry count (1..256). e0 < 0 marks an empty item (P <= p < Pmax).
+struct __align__(16) PairDesc {
+    int64_t e0;
+    int32_t l;
+    int32_t n;
+};
+
 struct AttnParams {
     const uint16_t* q;
     const uint16_t* k;
@@ -31,8 +40,7 @@ struct AttnParams {
     // past pairs
     const uint64_t* entries;
     const int64_t* segoff;      // list l spans entries [segoff[l*nch], segoff[(l+1)*nch])
-    const int64_t* tile_start;  // past pair prefix per list, tile_start[L] = P
-    const int64_t* item_list;   // list of each past pair (find_list precomputed), [Pmax]
+    const PairDesc* pairs;       // descriptor of each past pair, [Pmax]
     int64_t L, Pmax;
     uint16_t* opart;  // bf16 [B, Hq, N, kp, d]
     float* lpart;     // fp32 [B, Hq, N, kp]
@@ -56,13 +64,25 @@ __device__ __forceinline__ int64_t find_list(const int64_t* __restrict__ ts, int
     return lo;
 }
 
-// item_list[p] = find_list(p) for every past pair p < P, -1 for p in [P, Pmax): the attention
-// roles then decode an item with one load instead of a binary search of dependent loads.
-__global__ void __launch_bounds__(256) moba_item_list_kernel(const int64_t* __restrict__ ts, int64_t L, int64_t Pmax,
-                                                             int64_t* __restrict__ item_list) {
+// pairs[p] for every p < Pmax from the per-list pair prefix ts (ts[L] = P) and the list
+// bounds segoff (list l spans entries [segoff[l*nch], segoff[(l+1)*nch])).
+__global__ void __launch_bounds__(256) moba_item_list_kernel(const int64_t* __restrict__ ts,
+                                                             const int64_t* __restrict__ segoff, int64_t L,
+                                                             int64_t nch, int64_t Pmax, PairDesc* __restrict__ pairs) {
     const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (p >= Pmax) return;
-    item_list[p] = p < ts[L] ? find_list(ts, L, p) : -1;
+    PairDesc d;
+    d.e0 = -1;
+    d.l = 0;
+    d.n = 0;
+    if (p < ts[L]) {
+        const int64_t l = find_list(ts, L, p);
+        const int64_t le = segoff[(l + 1) * nch];
+        d.e0 = segoff[l * nch] + (p - ts[l]) * MOBA_PAIR_ROWS;
+        d.l = (int32_t)l;
+        d.n = (int32_t)((le - d.e0 < MOBA_PAIR_ROWS) ? le - d.e0 : MOBA_PAIR_ROWS);
+    }
+    pairs[p] = d;
 }
 
 struct TileInfo {
@@ -85,31 +105,37 @@ struct PairInfo {
     int64_t ns;  // K/V steps of the pair = the longer tile's steps
 };
 
-__device__ __forceinline__ PairInfo decode_pair(const AttnParams& a, int64_t item) {
+// The descriptor of an item (a dummy for own-block items, whose decoding is arithmetic only).
+__device__ __forceinline__ PairDesc pair_desc(const AttnParams& a, int64_t item) {
+    if (item < a.Pmax) return a.pairs[item];
+    PairDesc d;
+    d.e0 = -1;
+    d.l = 0;
+    d.n = 0;
+    return d;
+}
+
+__device__ __forceinline__ PairInfo decode_pair(const AttnParams& a, int64_t item, const PairDesc pd) {
     PairInfo pi;
     pi.t[0].kind = -1;
     pi.t[1].kind = -1;
     pi.ns = 0;
     if (item < a.Pmax) {
-        const int64_t P = a.tile_start[a.L];
-        if (item >= P) return pi;
-        const int64_t l = a.item_list[item];
-        const int64_t m = item - a.tile_start[l];
-        const int64_t ls = a.segoff[l * a.nch], le = a.segoff[(l + 1) * a.nch];
+        if (pd.e0 < 0) return pi;
+        const int64_t l = pd.l;
         const int64_t j = l % a.nblk;
         const int hk = (int)((l / a.nblk) % a.Hkv);
         const int b = (int)(l / (a.nblk * a.Hkv));
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
             TileInfo& ti = pi.t[x];
-            const int64_t e0 = ls + m * MOBA_PAIR_ROWS + x * MOBA_TILE;
-            if (e0 >= le) continue;
+            if (x * MOBA_TILE >= pd.n) continue;
             ti.kind = 0;
             ti.j = j;
             ti.hk = hk;
             ti.b = b;
-            ti.e0 = e0;
-            ti.ne = (le - e0 < MOBA_TILE) ? le - e0 : MOBA_TILE;
+            ti.e0 = pd.e0 + x * MOBA_TILE;
+            ti.ne = (pd.n - x * MOBA_TILE < MOBA_TILE) ? pd.n - x * MOBA_TILE : MOBA_TILE;
             ti.klo = j * a.bs;
             ti.khi = ti.klo + a.bs;
             ti.hq = 0;
@@ -149,4 +175,8 @@ __device__ __forceinline__ PairInfo decode_pair(const AttnParams& a, int64_t ite
     const int64_t n0 = tile_steps(pi.t[0]), n1 = tile_steps(pi.t[1]);
     pi.ns = n0 > n1 ? n0 : n1;
     return pi;
+}
+
+__device__ __forceinline__ PairInfo decode_pair(const AttnParams& a, int64_t item) {
+    return decode_pair(a, item, pair_desc(a, item));
 }

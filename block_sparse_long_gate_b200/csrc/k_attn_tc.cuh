@@ -15,15 +15,20 @@
 // shared memory feeds twice the MMA work.
 //
 // Roles (352 threads, one CTA per SM, persistent over the pairs):
-//   warp 0     producer: TMA loads of K steps into a 3-slot ring and of V steps
-//              into a 2-slot ring (3-D maps, 128-byte swizzle); K runs one step ahead
+//   warp 0     producer: lane 0 issues the TMA loads of K steps into a 3-slot ring
+//              and of V steps into a 2-slot ring (3-D maps, 128-byte swizzle; K runs
+//              one step ahead); the whole warp gathers each tile's Q rows (cp.async,
+//              swizzled) as soon as the previous tile of the same X has issued its
+//              last Q K^T, so a tile's rows arrive while the previous one finishes
 //   warp 1     MMA issuer of tile A (and TMEM owner), warp 10 MMA issuer of tile B.
 //              Per step i of a pair each issues [P V for step i-1, Q K^T for step i]
 //              of its tile; the two alternate whole iterations through turn barriers
 //              so the pipe runs one tile's batch, then the other's.
 //   warps 2-5  softmax of tile A; warps 6-9 softmax of tile B. Each thread owns one
-//              row: gathers its Q row (cp.async, swizzled), runs the softmax with a
-//              lazily moved maximum, and writes the normalised row in the epilogue.
+//              row: it runs the softmax with a lazily moved maximum and writes the
+//              normalised row in the epilogue.
+// Every role decodes an item from its 16-byte descriptor; the producer and the
+// issuers load it an item ahead.
 // TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512) (fp32, 128 lanes).
 // P_X (bf16 pairs) overwrites columns [64,128) of S_X once they have been read.
 // The running maximum used for P only moves when the row maximum grows by more
@@ -60,7 +65,8 @@ struct __align__(64) TcMaps {
 struct TcBars {
     uint64_t k_full[TC_KSLOTS], k_empty[TC_KSLOTS];
     uint64_t v_full[TC_VSLOTS], v_empty[TC_VSLOTS];
-    uint64_t q_full[2];   // per tile: its 128 softmax threads gathered their Q rows
+    uint64_t q_full[2];   // per tile: the producer warp's 32 lanes gathered its Q rows
+    uint64_t q_empty[2];  // per tile: its last Q K^T has completed (Q_X may be refilled)
     uint64_t s_full[2];   // per tile: Q K^T of a step is in S_X (and P V of the previous step in O_X)
     uint64_t p_full[2];   // per tile: P_X of a step is in TMEM
     uint64_t o_full[2];   // per tile: the tile's last P V is in O_X
@@ -235,6 +241,41 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, vol
 }
 
 
+// Identity of row r of a tile: its query token and head, and for a past tile the slot of
+// the partial (from the row's entry word en).
+struct QRow {
+    int64_t t;
+    int hq, slot;
+    bool valid;
+};
+
+__device__ __forceinline__ QRow q_row(const TileInfo& ti, uint64_t en, int r) {
+    QRow q;
+    if (ti.kind == 0) {
+        q.valid = r < ti.ne;
+        q.t = q.valid ? entry_t(en) : 0;
+        q.hq = q.valid ? entry_hq(en) : 0;
+        q.slot = q.valid ? entry_slot(en) : 0;
+    } else {
+        q.valid = r < ti.nt;
+        q.t = ti.t0 + r;
+        q.hq = ti.hq;
+        q.slot = 0;
+    }
+    return q;
+}
+
+// Requests row r of a tile's Q into the swizzled tile (q_dst: the row's 128-byte line; 16-byte
+// chunks XOR-swizzled by r & 7, the two 64-feature halves 16 KB apart). Rows past the tile's
+// end are zero-filled. The caller waits for the copies.
+__device__ __forceinline__ void gather_q_row(const AttnParams& a, const TileInfo& ti, const QRow& qr,
+                                             uint32_t q_dst, int r) {
+    const uint16_t* src = a.q + (qr.valid ? (((int64_t)ti.b * a.N + qr.t) * a.Hq + qr.hq) * MOBA_D : 0);
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+        cp_async_16_zfill(q_dst + (c >> 3) * 16384 + (((c & 7) ^ (r & 7)) << 4), src + c * 8, qr.valid);
+}
+
 __global__ void __launch_bounds__(TC_THREADS, 1)
     moba_attn_tc_kernel(const AttnParams a, const __grid_constant__ TcMaps maps, int64_t items) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -261,7 +302,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             bars->v_issued[s] = 0;
         }
         for (int x = 0; x < 2; ++x) {
-            mbar_init(&bars->q_full[x], 128);
+            mbar_init(&bars->q_full[x], 32);
+            mbar_init(&bars->q_empty[x], 1);
             mbar_init(&bars->s_full[x], 1);
             mbar_init(&bars->p_full[x], 128);
             mbar_init(&bars->o_full[x], 1);
@@ -289,46 +331,84 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const uint32_t tmem = bars->tmem_base;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            uint32_t gk = 0, gv = 0;  // K and V steps issued so far
-            bool ok = true;
-            auto load = [&](bool is_v, int hk, int row) -> bool {
-                const uint32_t g = is_v ? gv : gk;
-                const uint32_t nslots = is_v ? TC_VSLOTS : TC_KSLOTS;
-                const uint32_t s = g % nslots;
-                uint64_t* full = is_v ? &bars->v_full[s] : &bars->k_full[s];
-                uint64_t* empty = is_v ? &bars->v_empty[s] : &bars->k_empty[s];
-                // completion #(g/n - 1) of the slot's empty barrier; #(g/n - 2) was waited n loads ago
-                if (!tc_wait(empty, ((g / nslots) & 1) ^ 1, abort_flag, true)) return false;
-                uint8_t* dst = (is_v ? sV : sK) + s * TC_STEP_BYTES;
-                const void* map = is_v ? (const void*)&maps.v : (const void*)&maps.k;
-                mbar_arrive_expect_tx(full, TC_STEP_BYTES);
-                tma_load_3d(smem_u32(dst), map, full, 0, hk, row);
-                tma_load_3d(smem_u32(dst + 16384), map, full, 64, hk, row);
-                if (is_v) {
-                    bars->v_issued[s] += 1;
-                    ++gv;
-                } else {
-                    bars->k_issued[s] += 1;
-                    ++gk;
+        // ------------------------------------------------------------ producer warp
+        // Lane 0 streams K and V. All 32 lanes gather Q: lane l takes rows l, l + 32, l + 64 and
+        // l + 96 of a tile. An item's tiles are gathered after its first K step is requested and
+        // before its first V step: the tile's first Q K^T needs Q and K0, its first P V comes
+        // after a softmax. The entry words of the item's rows are loaded when the item starts.
+        uint32_t gk = 0, gv = 0;  // K and V steps issued (lane 0)
+        uint32_t nq[2] = {0, 0};  // tiles of A and of B gathered so far
+        bool ok = true;
+        auto load = [&](bool is_v, int hk, int row) -> bool {  // lane 0 only
+            const uint32_t g = is_v ? gv : gk;
+            const uint32_t nslots = is_v ? TC_VSLOTS : TC_KSLOTS;
+            const uint32_t s = g % nslots;
+            uint64_t* full = is_v ? &bars->v_full[s] : &bars->k_full[s];
+            uint64_t* empty = is_v ? &bars->v_empty[s] : &bars->k_empty[s];
+            // completion #(g/n - 1) of the slot's empty barrier; #(g/n - 2) was waited n loads ago
+            if (!tc_wait(empty, ((g / nslots) & 1) ^ 1, abort_flag, true)) return false;
+            uint8_t* dst = (is_v ? sV : sK) + s * TC_STEP_BYTES;
+            const void* map = is_v ? (const void*)&maps.v : (const void*)&maps.k;
+            mbar_arrive_expect_tx(full, TC_STEP_BYTES);
+            tma_load_3d(smem_u32(dst), map, full, 0, hk, row);
+            tma_load_3d(smem_u32(dst + 16384), map, full, 64, hk, row);
+            if (is_v) {
+                bars->v_issued[s] += 1;
+                ++gv;
+            } else {
+                bars->k_issued[s] += 1;
+                ++gk;
+            }
+            return true;
+        };
+        PairDesc dn = pair_desc(a, blockIdx.x);
+        for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x) {
+            const PairDesc d = dn;
+            if (item + gridDim.x < items) dn = pair_desc(a, item + gridDim.x);  // an item ahead
+            const PairInfo pi = decode_pair(a, item, d);
+            if (pi.ns == 0) continue;
+            uint64_t ew[2][4];  // entry words of this lane's rows (past tiles)
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int rr = lane + 32 * k;
+                    ew[x][k] = (pi.t[x].kind == 0 && rr < pi.t[x].ne) ? a.entries[pi.t[x].e0 + rr] : 0ull;
                 }
-                return true;
-            };
-            for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x) {
-                const PairInfo pi = decode_pair(a, item);
-                if (pi.ns == 0) continue;
-                const bool first = pi.t[0].kind >= 0;
-                const int hk = first ? pi.t[0].hk : pi.t[1].hk;
-                const int64_t row0 = (int64_t)(first ? pi.t[0].b : pi.t[1].b) * a.N + (first ? pi.t[0].klo : pi.t[1].klo);
-                // K one step ahead of V: K0, K1, V0, K2, V1, ...
-                if (!(ok = load(false, hk, (int)row0))) break;
+            const bool first = pi.t[0].kind >= 0;
+            const int hk = first ? pi.t[0].hk : pi.t[1].hk;
+            const int64_t row0 = (int64_t)(first ? pi.t[0].b : pi.t[1].b) * a.N + (first ? pi.t[0].klo : pi.t[1].klo);
+            if (lane == 0) ok = load(false, hk, (int)row0);  // K0
+            if (!(ok = __shfl_sync(0xffffffffu, ok, 0))) break;
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const TileInfo& ti = pi.t[x];
+                if (ti.kind < 0) continue;
+                // completion #nq-1 of q_empty[x]: the previous tile of x has read Q_x for the last
+                // time (for the first tile the wait returns at once); #nq-2 was waited before the
+                // previous gather
+                if (!(ok = tc_wait_warp(&bars->q_empty[x], (nq[x] & 1) ^ 1, abort_flag))) break;
+                const uint32_t base = smem_u32(sQ + x * TC_Q_BYTES);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int rr = lane + 32 * k;
+                    gather_q_row(a, ti, q_row(ti, ew[x][k], rr), base + rr * 128, rr);
+                }
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                mbar_arrive(&bars->q_full[x]);
+                ++nq[x];
+            }
+            if (!ok) break;
+            if (lane == 0) {  // K one step ahead of V: K0, K1, V0, K2, V1, ...
                 for (int64_t i = 0; i < pi.ns; ++i) {
                     if (i + 1 < pi.ns && !(ok = load(false, hk, (int)(row0 + (i + 1) * MOBA_KCHUNK)))) break;
                     if (!(ok = load(true, hk, (int)(row0 + i * MOBA_KCHUNK)))) break;
                 }
             }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
         }
+        cp_async_wait_all();  // no copy may still write the shared memory when the CTA leaves
         __syncwarp();
     } else if (warp == 1 || warp == TC_THREADS / 32 - 1) {
         // ------------------------------------------------------------ MMA issuers
@@ -352,8 +432,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         uint32_t px = 0, tx = 0;  // P V steps issued, tiles finished
         uint32_t it = 0;          // iterations of the issue loop (the same sequence for both issuers)
         bool ok = true;
+        PairDesc dn = pair_desc(a, blockIdx.x);
         for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x) {
-            const PairInfo pi = decode_pair(a, item);
+            const PairDesc d = dn;
+            if (item + gridDim.x < items) dn = pair_desc(a, item + gridDim.x);  // an item ahead
+            const PairInfo pi = decode_pair(a, item, d);
             if (pi.ns == 0) continue;
             const int64_t nx = tile_steps(x ? pi.t[1] : pi.t[0]);
             // completion #tx of q_full[x]: #tx-1 was waited for the previous tile of x
@@ -400,6 +483,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         tc_mma_ss_w(tS, dq + off, kd + off, idesc_qk, k > 0 ? 1u : 0u);
                     }
                     tc_commit_w(&bars->s_full[x]);
+                    if (i + 1 == nx) tc_commit_w(&bars->q_empty[x]);  // the tile's last read of Q_x
                 }
                 mbar_arrive_w(&bars->turn[x ^ 1]);
                 ++it;
@@ -427,7 +511,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
         const uint32_t tS = tmem + x * 128 + lane_off;
         const uint32_t tO = tmem + 256 + x * 128 + lane_off;
-        uint8_t* sQx = sQ + x * TC_Q_BYTES;
         uint32_t g = 0, tile_i = 0;
         for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
             const PairInfo pi = decode_pair(a, item);
@@ -450,18 +533,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 valid = r < ti.nt;
                 t = ti.t0 + r;
                 hq = ti.hq;
-            }
-            // gather this row of Q into the swizzled tile (zero rows past the end). The buffer is
-            // free: the previous tile's epilogue waited for its last P V, after every Q K^T of it.
-            {
-                const uint16_t* src = a.q + (valid ? (((int64_t)ti.b * a.N + t) * a.Hq + hq) * MOBA_D : 0);
-                const uint32_t dst = smem_u32(sQx) + r * 128;
-#pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    cp_async_16_zfill(dst + (c >> 3) * 16384 + (((c & 7) ^ (r & 7)) << 4), src + c * 8, valid);
-                cp_async_wait_all();
-                fence_proxy_async_smem();
-                mbar_arrive(&bars->q_full[x]);
             }
             // last key column this row may read, relative to the tile's first key: the key range
             // and, on the own block, causality (u <= t)

@@ -105,6 +105,7 @@ int make_plan(int B, int Hq, int Hkv, int64_t N, int d, int bs, int topk, Plan* 
     if (P.nblk > MOBA_MAX_BLOCKS) return MOBA_ERR_SHAPE;  // per-block counters live in shared memory
     P.nfull = N / bs;
     P.L = (int64_t)B * Hkv * P.nblk;
+    if (P.L >= ((int64_t)1 << 31)) return MOBA_ERR_SHAPE;  // a pair descriptor holds its list in 32 bits
     P.nch = cdiv(N, INV_CHUNK);
     // exact number of earlier-block selections of well-formed rows: sum_t min(c(t), k - 1)
     int64_t per_head = 0;
@@ -147,7 +148,7 @@ int make_plan(int B, int Hq, int Hkv, int64_t N, int d, int bs, int topk, Plan* 
     P.off_entries = o;
     o = align256(o + sizeof(uint64_t) * (size_t)(P.E > 0 ? P.E : 1));
     P.off_items = o;
-    o = align256(o + sizeof(int64_t) * (size_t)(P.Pmax > 0 ? P.Pmax : 1));
+    o = align256(o + sizeof(PairDesc) * (size_t)(P.Pmax > 0 ? P.Pmax : 1));
     P.off_opart = o;
     o = align256(o + sizeof(uint16_t) * (size_t)B * Hq * N * (P.kp > 0 ? P.kp : 1) * MOBA_D);
     P.off_lpart = o;
@@ -302,7 +303,7 @@ int run_invert(const Plan& P, const int32_t* idx, char* ws, cudaStream_t st) {
     if ((rc = run_scan(s2, P.L, parts, tiles, st))) return rc;
     if (P.Pmax > 0) {
         moba_item_list_kernel<<<(unsigned)cdiv(P.Pmax, SCAN_THREADS), SCAN_THREADS, 0, st>>>(
-            tiles, P.L, P.Pmax, (int64_t*)(ws + P.off_items));
+            tiles, segoff, P.L, P.nch, P.Pmax, (PairDesc*)(ws + P.off_items));
         count_launch();
         if ((rc = launch_ok())) return rc;
     }
@@ -330,8 +331,7 @@ AttnParams attn_params(const Plan& P, const void* q, const void* k, const void* 
     a.nch = P.nch;
     a.entries = ws ? (const uint64_t*)(ws + P.off_entries) : nullptr;
     a.segoff = ws ? (const int64_t*)(ws + P.off_segoff) : nullptr;
-    a.tile_start = ws ? (const int64_t*)(ws + P.off_tiles) : nullptr;
-    a.item_list = ws ? (const int64_t*)(ws + P.off_items) : nullptr;
+    a.pairs = ws ? (const PairDesc*)(ws + P.off_items) : nullptr;
     a.L = P.L;
     a.Pmax = P.Pmax;
     a.opart = ws ? (uint16_t*)(ws + P.off_opart) : nullptr;
