@@ -9,27 +9,44 @@
 // of a hybrid model ("KIMI MoBA" blog, section 3, hybrid_layers; the pages run
 // decode with full attention) keeps every block.
 //
-// Three kernels:
-//   select  one CTA per (b, kv head): exact fp64 scores of the G query heads
-//           against the cached block summaries Kbar, top-k per head, then the
-//           union of the group's kept blocks with a G-bit mask per block (the
-//           heads that kept it), so each K/V block is read once for the group;
-//   attend  one CTA per (b, kv head, union entry, 512-key chunk): streams the
-//           chunk's keys and values through shared memory once and keeps an
-//           online softmax (max, sum, 128 outputs) for every head that kept the
-//           block; writes one partial per head;
-//   merge   one CTA per (b, query head): log-sum-exp merge of its partials.
+// Four kernels:
+//   select  one CTA per query head: exact fp64 scores against the cached block
+//           summaries Kbar into shared memory; each warp picks the best topk - 1
+//           of a quarter of the blocks by rounds of a warp arg-max over per-lane
+//           maxima (only the lane that lost its maximum rescans), and warp 0 picks
+//           the head's topk - 1 among the four lists the same way;
+//   union   one CTA per (b, kv head): the union of the group's kept blocks in
+//           ascending order with a G-bit mask per block (the heads that kept it),
+//           so each K/V block is read once for the whole group;
+//   attend  one CTA per (b, kv head, union entry, 512-key chunk), four warps of
+//           128 keys each. A warp streams its keys and values through its own
+//           3-stage cp.async ring of 16-key stages and runs both products on the
+//           tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the
+//           group's heads as the 16 rows: S = Q K^T, an online softmax per row,
+//           O += P V. The four warps' states are combined in shared memory into
+//           one partial per head that kept the block;
+//   merge   one CTA per (b, query head): log-sum-exp merge of its partials, the
+//           warps splitting the partials.
 // Memory bound: the K/V bytes of the union blocks dominate.
 #pragma once
 #include "common.cuh"
 
-#define DEC_THREADS 128
-#define DEC_CHUNK 512       // keys per attend CTA
-#define DEC_TILE 64         // keys per shared-memory tile
-#define DEC_MAX_G 16        // query heads per kv head (static shared memory of the attend kernel)
-#define DEC_PART (MOBA_D + 2)  // one partial: m (log2 units), l, o[128]
-#define DEC_KSTRIDE (MOBA_D + 2)  // K tile row stride in bf16: 65 words, so lanes reading one feature
-                                  // of 32 different keys hit 32 different banks
+#define DEC_MAX_G 16        // query heads per kv head: the 16 rows of an m16n8k16 product
+#define DEC_SEL_THREADS 128
+#define DEC_UNION_THREADS 256
+#define DEC_WARPS 4
+#define DEC_CHUNK 512                               // keys per attend CTA
+#define DEC_WARP_KEYS (DEC_CHUNK / DEC_WARPS)       // keys per warp
+#define DEC_SKEYS 16                                // keys per ring stage
+#define DEC_STAGES 3
+#define DEC_ROW 272  // bytes per staged key row: 256 + 16, so the 8 rows one ldmatrix reads hit distinct banks
+#define DEC_STAGE_BYTES (2 * DEC_SKEYS * DEC_ROW)   // K rows, then V rows
+#define DEC_ATTEND_SMEM (DEC_WARPS * DEC_STAGES * DEC_STAGE_BYTES)
+#define DEC_MERGE_THREADS 256
+#define DEC_PART 132  // one partial: m (log2 units), l, 2 unused, o[128] (16-byte aligned)
+
+static_assert(DEC_WARPS * 32 == MOBA_D, "the combine gives each thread one output feature");
+static_assert(DEC_WARPS * DEC_MAX_G * (MOBA_D + 2) * 4 <= DEC_ATTEND_SMEM, "combine area exceeds the rings");
 
 struct DecodeParams {
     const uint16_t* q;    // [B, Hq, d]
@@ -43,6 +60,7 @@ struct DecodeParams {
     int64_t umax;         // union capacity per (b, kv head)
     int64_t nch;          // chunks per block
     int full;             // keep every block
+    int32_t* kept;        // [B*Hkv][G][max(topk - 1, 1)] kept earlier blocks per head, ascending
     int32_t* ucount;      // [B*Hkv]
     int32_t* ulist;       // [B*Hkv][umax] block ids, ascending
     uint32_t* umask;      // [B*Hkv][umax] heads of the group that kept the block
@@ -53,140 +71,233 @@ struct DecodeParams {
     float scale_log2;     // log2(e) / sqrt(d)
 };
 
+// (score desc, block asc): does (s2, j2) rank before (s, j)? A NaN score never ranks first.
+__device__ __forceinline__ bool dec_before(double s2, int32_t j2, double s, int32_t j) {
+    return s2 > s || (s2 == s && j2 < j);
+}
+
+// Warp arg-max of (s, j) by dec_before; every lane gets the winner.
+__device__ __forceinline__ void dec_warp_best(double& s, int32_t& j) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        const int32_t j2 = __shfl_xor_sync(0xffffffffu, j, o);
+        if (dec_before(s2, j2, s, j)) {
+            s = s2;
+            j = j2;
+        }
+    }
+}
+
+// Rounds of a warp arg-max over the n scores sc[0 .. n) with block ids jd[i] (i itself when jd
+// is null): lane l owns entries l, l + 32, ...; each round's winner is struck out (set to NaN,
+// which never ranks first) and only its owner rescans. Lane 0 writes up to `want` winners in
+// rank order to ws / wj; returns their number (the same on every lane).
+__device__ __forceinline__ int dec_rounds(double* sc, const int32_t* jd, int n, int want, double* ws, int32_t* wj,
+                                          int lane) {
+    double lb = -INFINITY;
+    int32_t lj = 0x7FFFFFFF;
+    int li = -1;
+    auto rescan = [&]() {
+        lb = -INFINITY;
+        lj = 0x7FFFFFFF;
+        li = -1;
+        for (int i = lane; i < n; i += 32) {
+            const double s = sc[i];
+            const int32_t j = jd ? jd[i] : i;
+            if (dec_before(s, j, lb, lj)) {
+                lb = s;
+                lj = j;
+                li = i;
+            }
+        }
+    };
+    rescan();
+    int got = 0;
+    for (; got < want; ++got) {
+        double bs = lb;
+        int32_t bj = lj;
+        dec_warp_best(bs, bj);
+        if (bj == 0x7FFFFFFF) break;  // nothing left
+        if (lane == 0) {
+            ws[got] = bs;
+            wj[got] = bj;
+        }
+        if (li >= 0 && lj == bj) {  // this lane owned the winner
+            sc[li] = __longlong_as_double(0x7FF8000000000000ll);
+            rescan();
+        }
+        __syncwarp();
+    }
+    return got;
+}
+
 // ---------------------------------------------------------------- select
-// dynamic smem: c doubles (scores of one head) + G * topk ints (kept blocks per head)
-__global__ void __launch_bounds__(DEC_THREADS) moba_decode_select_kernel(const DecodeParams p) {
+// grid (G, Hkv, B); dynamic smem (when c > topk - 1 > 0): the c scores, then two areas of 4 (topk - 1)
+// (score, block) candidates: the four warps' lists and their compacted merge.
+__global__ void __launch_bounds__(DEC_SEL_THREADS) moba_decode_select_kernel(const DecodeParams p) {
     extern __shared__ __align__(16) uint8_t smem[];
-    const int hk = blockIdx.x, b = blockIdx.y;
+    __shared__ double sq[MOBA_D];
+    __shared__ int32_t cnt[DEC_SEL_THREADS / 32];
+    __shared__ double fs[MOBA_MAX_TOPK];
+    __shared__ int32_t fj[MOBA_MAX_TOPK];
+    const int g = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int hq = hk * p.G + g;
+    const int64_t bh = (int64_t)b * p.Hkv + hk;
     const int64_t c = p.c;
     const int kp = p.topk - 1;
-    const int64_t bh0 = (int64_t)blockIdx.y * p.Hkv + blockIdx.x;
-    if (p.full) {  // every block 0 .. c is kept by every head
-        const uint32_t all = (1u << p.G) - 1u;
-        for (int64_t j = threadIdx.x; j <= c; j += DEC_THREADS) {
-            p.ulist[bh0 * p.umax + j] = (int32_t)j;
-            p.umask[bh0 * p.umax + j] = all;
-        }
-        if (threadIdx.x == 0) p.ucount[bh0] = (int32_t)(c + 1);
-        return;
-    }
-    const int64_t npast = c < kp ? c : kp;  // earlier blocks kept per head
-    double* sc = (double*)smem;
-    int32_t* kept = (int32_t*)(smem + sizeof(double) * (c > 0 ? c : 1));  // [G][npast]
-    __shared__ double rs[DEC_THREADS / 32];
-    __shared__ int32_t rj[DEC_THREADS / 32];
+    const int npast = (int)(c < kp ? c : kp);  // earlier blocks kept
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t bh = (int64_t)b * p.Hkv + hk;
-
-    for (int g = 0; g < p.G; ++g) {
-        const int hq = hk * p.G + g;
-        int32_t* kg = kept + (int64_t)g * (npast > 0 ? npast : 1);
-        if (c <= kp) {  // every earlier block is kept
-            for (int64_t j = threadIdx.x; j < npast; j += DEC_THREADS) kg[j] = (int32_t)j;
-            continue;
-        }
-        // exact fp64 scores <q, Kbar_j>, features ascending (one fused multiply-add each)
+    int32_t* kept = p.kept + (bh * p.G + g) * (kp > 0 ? kp : 1);
+    if (c > kp && kp > 0) {
+        double* sc = (double*)smem;                  // [c] scores
+        double* cs = sc + c;                         // [4][kp] candidate scores per warp
+        double* ms = cs + 4 * kp;                    // [4 kp] the compacted candidates
+        int32_t* cj = (int32_t*)(ms + 4 * kp);       // [4][kp] candidate blocks per warp
+        int32_t* mj = cj + 4 * kp;                   // [4 kp]
         const uint16_t* qr = p.q + ((int64_t)b * p.Hq + hq) * MOBA_D;
-        for (int64_t j = threadIdx.x; j < c; j += DEC_THREADS) {
+        for (int e = threadIdx.x; e < MOBA_D; e += DEC_SEL_THREADS) sq[e] = (double)bf16_bits_to_float(qr[e]);
+        __syncthreads();
+        // exact fp64 scores <q, Kbar_j>, features ascending (one fused multiply-add each); a NaN
+        // score ranks as -inf
+        for (int64_t j = threadIdx.x; j < c; j += DEC_SEL_THREADS) {
             const double* kb = p.kbar + (bh * p.kbar_rows + j) * MOBA_D;
             double s = 0.0;
 #pragma unroll 8
-            for (int e = 0; e < MOBA_D; ++e) s = fma((double)bf16_bits_to_float(qr[e]), kb[e], s);
-            sc[j] = s;
+            for (int e = 0; e < MOBA_D; ++e) s = fma(sq[e], kb[e], s);
+            sc[j] = (s == s) ? s : -INFINITY;
         }
         __syncthreads();
-        // kp rounds of a block-wide arg-max over (score desc, index asc); the winner is struck out
-        for (int r = 0; r < kp; ++r) {
-            double best = -INFINITY;
-            int32_t bj = 0x7FFFFFFF;
-            for (int64_t j = threadIdx.x; j < c; j += DEC_THREADS) {
-                const double s = sc[j];
-                if (s > best || (s == best && (int32_t)j < bj)) {
-                    best = s;
-                    bj = (int32_t)j;
+        // each warp: the best kp of its quarter of the blocks
+        const int lo = (int)(c * warp / 4), hi = (int)(c * (warp + 1) / 4);
+        const int n = dec_rounds(sc + lo, nullptr, hi - lo, kp, cs + warp * kp, cj + warp * kp, lane);
+        __syncwarp();
+        if (lane == 0) {
+            for (int i = 0; i < n; ++i) cj[warp * kp + i] += lo;  // block ids
+            cnt[warp] = n;
+        }
+        __syncthreads();
+        if (warp == 0) {  // the head's best kp among the four lists, by the same rounds
+            int off = 0;
+            for (int w = 0; w < 4; ++w) {
+                for (int i = lane; i < cnt[w]; i += 32) {
+                    ms[off + i] = cs[w * kp + i];
+                    mj[off + i] = cj[w * kp + i];
                 }
+                off += cnt[w];
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const double s2 = __shfl_xor_sync(0xffffffffu, best, o);
-                const int32_t j2 = __shfl_xor_sync(0xffffffffu, bj, o);
-                if (s2 > best || (s2 == best && j2 < bj)) {
-                    best = s2;
-                    bj = j2;
-                }
+            __syncwarp();
+            const int m = dec_rounds(ms, mj, off, kp, fs, fj, lane);
+            __syncwarp();
+            // ascending block order: winner i goes to its rank among the m winners
+            for (int i = lane; i < m; i += 32) {
+                int rank = 0;
+                for (int t = 0; t < m; ++t) rank += fj[t] < fj[i];
+                kept[rank] = fj[i];
             }
-            if (lane == 0) {
-                rs[warp] = best;
-                rj[warp] = bj;
-            }
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                for (int w = 1; w < DEC_THREADS / 32; ++w)
-                    if (rs[w] > best || (rs[w] == best && rj[w] < bj)) {
-                        best = rs[w];
-                        bj = rj[w];
-                    }
-                kg[r] = bj;
-                sc[bj] = -INFINITY;  // struck out (real scores are finite)
-            }
-            __syncthreads();
         }
+    } else {
+        for (int j = threadIdx.x; j < npast; j += DEC_SEL_THREADS) kept[j] = j;  // every earlier block
     }
-    __syncthreads();
-    if (threadIdx.x != 0) return;
-    // per head: ascending kept blocks (own block last) into idx_out, then the union of the group
-    for (int g = 0; g < p.G; ++g) {
-        int32_t* kg = kept + (int64_t)g * (npast > 0 ? npast : 1);
-        for (int64_t i = 1; i < npast; ++i) {  // insertion sort (npast <= topk - 1)
-            const int32_t x = kg[i];
-            int64_t u = i;
-            while (u > 0 && kg[u - 1] > x) {
-                kg[u] = kg[u - 1];
-                --u;
-            }
-            kg[u] = x;
-        }
-        if (p.idx_out) {
-            int32_t* orow = p.idx_out + ((int64_t)b * p.Hq + hk * p.G + g) * p.topk;
-            for (int i = 0; i < p.topk; ++i) orow[i] = i < npast ? kg[i] : (i == npast ? (int32_t)c : -1);
-        }
+    if (p.idx_out) {
+        __syncthreads();
+        int32_t* orow = p.idx_out + ((int64_t)b * p.Hq + hq) * p.topk;
+        for (int i = threadIdx.x; i < p.topk; i += DEC_SEL_THREADS)
+            orow[i] = i < npast ? kept[i] : (i == npast ? (int32_t)c : -1);
     }
-    // union: a G-way merge of the sorted lists, then the own block
+}
+
+// ---------------------------------------------------------------- union
+// grid (Hkv, B); dynamic smem: c masks. The blocks kept by any head of the group, ascending,
+// with the mask of the heads that kept each, then the own block c (kept by every head).
+__global__ void __launch_bounds__(DEC_UNION_THREADS) moba_decode_union_kernel(const DecodeParams p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ int32_t wsum[DEC_UNION_THREADS / 32];
+    const int hk = blockIdx.x, b = blockIdx.y;
+    const int64_t bh = (int64_t)b * p.Hkv + hk;
+    const int64_t c = p.c;
+    const uint32_t all = (1u << p.G) - 1u;  // G <= 16
     int32_t* ul = p.ulist + bh * p.umax;
     uint32_t* um = p.umask + bh * p.umax;
-    int64_t n = 0;
-    int64_t pos[DEC_MAX_G];
-    for (int g = 0; g < p.G; ++g) pos[g] = 0;
-    for (;;) {
-        int32_t j = 0x7FFFFFFF;
-        for (int g = 0; g < p.G; ++g)
-            if (pos[g] < npast) {
-                const int32_t x = kept[(int64_t)g * npast + pos[g]];
-                if (x < j) j = x;
-            }
-        if (j == 0x7FFFFFFF) break;
-        uint32_t mask = 0;
-        for (int g = 0; g < p.G; ++g)
-            if (pos[g] < npast && kept[(int64_t)g * npast + pos[g]] == j) {
-                mask |= 1u << g;
-                ++pos[g];
-            }
-        ul[n] = j;
-        um[n] = mask;
-        ++n;
+    if (p.full) {  // every block 0 .. c, kept by every head
+        for (int64_t j = threadIdx.x; j <= c; j += DEC_UNION_THREADS) {
+            ul[j] = (int32_t)j;
+            um[j] = all;
+        }
+        if (threadIdx.x == 0) p.ucount[bh] = (int32_t)(c + 1);
+        return;
     }
-    ul[n] = (int32_t)c;  // the own block, kept by every head
-    um[n] = (1u << p.G) - 1u;
-    ++n;
-    p.ucount[bh] = (int32_t)n;
+    uint32_t* mk = (uint32_t*)smem;  // [c]
+    const int kp = p.topk - 1;
+    const int kw = kp > 0 ? kp : 1;
+    const int npast = (int)(c < kp ? c : kp);
+    for (int64_t j = threadIdx.x; j < c; j += DEC_UNION_THREADS) mk[j] = 0u;
+    __syncthreads();
+    const int32_t* kept = p.kept + bh * p.G * kw;
+    for (int i = threadIdx.x; i < p.G * npast; i += DEC_UNION_THREADS) {
+        const int g = i / npast, r = i % npast;
+        atomicOr(&mk[kept[(int64_t)g * kw + r]], 1u << g);
+    }
+    __syncthreads();
+    // compaction in index order: thread t takes the contiguous range [t c / T, (t + 1) c / T)
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int64_t lo = c * t / DEC_UNION_THREADS, hi = c * (t + 1) / DEC_UNION_THREADS;
+    int n = 0;
+    for (int64_t j = lo; j < hi; ++j) n += mk[j] != 0u;
+    int incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int pos = incl - n;
+    for (int w = 0; w < warp; ++w) pos += wsum[w];
+    for (int64_t j = lo; j < hi; ++j)
+        if (mk[j] != 0u) {
+            ul[pos] = (int32_t)j;
+            um[pos] = mk[j];
+            ++pos;
+        }
+    if (t == DEC_UNION_THREADS - 1) {  // pos is now the number of earlier blocks in the union
+        ul[pos] = (int32_t)c;
+        um[pos] = all;
+        p.ucount[bh] = pos + 1;
+    }
 }
 
 // ---------------------------------------------------------------- attend
-// grid (umax * nch, Hkv, B); static smem: K and V tiles, the heads' queries, scores and state.
-// GM >= G (query heads per kv head) is a template argument so each thread's outputs stay in
-// registers; heads g >= G are never in a block's mask and are skipped.
-template <int GM>
-__global__ void __launch_bounds__(DEC_THREADS) moba_decode_attend_kernel(const DecodeParams p) {
+__device__ __forceinline__ void dec_ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void dec_ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+// D += A B, m16n8k16, A row-major bf16 (4 registers), B column-major bf16 (2), D fp32 (4)
+__device__ __forceinline__ void dec_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void dec_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void dec_wait_group() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// grid (umax * nch, Hkv, B), DEC_WARPS warps; dynamic smem DEC_ATTEND_SMEM.
+// Fragments of m16n8k16 (g8 = lane / 4, t4 = lane % 4): A rows g8 and g8 + 8, columns 2 t4 (+1)
+// and 2 t4 + 8 (+1); B column g8, rows 2 t4 (+1) and 2 t4 + 8 (+1); C rows g8 and g8 + 8,
+// columns 2 t4 (+1). The rows are the group's heads, zero beyond G.
+__global__ void __launch_bounds__(DEC_WARPS * 32, 2) moba_decode_attend_kernel(const DecodeParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
     const int hk = blockIdx.y, b = blockIdx.z;
     const int64_t bh = (int64_t)b * p.Hkv + hk;
     const int64_t u = blockIdx.x / p.nch, ch = blockIdx.x % p.nch;
@@ -196,140 +307,241 @@ __global__ void __launch_bounds__(DEC_THREADS) moba_decode_attend_kernel(const D
     const int64_t bend = (j == p.c) ? p.L : (j + 1) * p.bs;  // keys [j*bs, bend)
     const int64_t k0 = j * p.bs + ch * DEC_CHUNK;
     const int64_t k1 = (k0 + DEC_CHUNK < bend) ? k0 + DEC_CHUNK : bend;
-
-    __shared__ __align__(16) uint16_t sk[DEC_TILE][DEC_KSTRIDE];
-    __shared__ __align__(16) uint16_t sv[DEC_TILE][MOBA_D];
-    __shared__ float sq[GM][MOBA_D];
-    __shared__ float sp[GM][DEC_TILE];
-    __shared__ float sm[GM], sl[GM], sa[GM];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g8 = lane >> 2, t4 = lane & 3;
     const int G = p.G;
-    for (int i = threadIdx.x; i < G * MOBA_D; i += DEC_THREADS) {
-        const int g = i / MOBA_D, e = i % MOBA_D;
-        sq[g][e] = bf16_bits_to_float(p.q[((int64_t)b * p.Hq + hk * G + g) * MOBA_D + e]);
-    }
-    if (threadIdx.x < G) {
-        sm[threadIdx.x] = -INFINITY;
-        sl[threadIdx.x] = 0.f;
-    }
-    float o[GM];  // this thread's output feature e = threadIdx.x, per head
+    // this warp's keys [kw0, kw1), in stages of 16
+    const int64_t kw0 = k0 + warp * DEC_WARP_KEYS;
+    const int64_t kw1 = (kw0 + DEC_WARP_KEYS < k1) ? kw0 + DEC_WARP_KEYS : (k1 > kw0 ? k1 : kw0);
+    const int nst = (int)((kw1 - kw0 + DEC_SKEYS - 1) / DEC_SKEYS);
+
+    // Q as A fragments, 8 steps of 16 features
+    uint32_t qa[8][4];
+    {
+        const uint16_t* qb = p.q + ((int64_t)b * p.Hq + (int64_t)hk * G) * MOBA_D;
 #pragma unroll
-    for (int g = 0; g < GM; ++g) o[g] = 0.f;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int64_t t0 = k0; t0 < k1; t0 += DEC_TILE) {
-        const int nk = (int)((k1 - t0 < DEC_TILE) ? k1 - t0 : DEC_TILE);
-        __syncthreads();  // the previous tile is no longer read
-        for (int i = threadIdx.x; i < DEC_TILE * (MOBA_D / 8); i += DEC_THREADS) {
-            const int kk = i / (MOBA_D / 8), c8 = i % (MOBA_D / 8);
-            uint4 kw = make_uint4(0u, 0u, 0u, 0u), vw = kw;
-            if (kk < nk) {
-                const int64_t row = ((int64_t)b * p.Lmax + t0 + kk) * p.Hkv + hk;
-                kw = ld_nc_v4(p.k + row * MOBA_D + c8 * 8);
-                vw = ld_nc_v4(p.v + row * MOBA_D + c8 * 8);
-            }
-            uint32_t* kd = reinterpret_cast<uint32_t*>(&sk[kk][c8 * 8]);  // 4-byte aligned rows
-            kd[0] = kw.x;
-            kd[1] = kw.y;
-            kd[2] = kw.z;
-            kd[3] = kw.w;
-            *reinterpret_cast<uint4*>(&sv[kk][c8 * 8]) = vw;
+        for (int ks = 0; ks < 8; ++ks) {
+            const int f = ks * 16 + 2 * t4;
+            qa[ks][0] = g8 < G ? *reinterpret_cast<const uint32_t*>(qb + g8 * MOBA_D + f) : 0u;
+            qa[ks][1] = g8 + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (g8 + 8) * MOBA_D + f) : 0u;
+            qa[ks][2] = g8 < G ? *reinterpret_cast<const uint32_t*>(qb + g8 * MOBA_D + f + 8) : 0u;
+            qa[ks][3] = g8 + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (g8 + 8) * MOBA_D + f + 8) : 0u;
         }
-        __syncthreads();
-        // scores: thread (kk = t % 64) for heads g = t / 64, t / 64 + 2, ...
+    }
+    uint8_t* ring = smem + warp * (DEC_STAGES * DEC_STAGE_BYTES);
+    // stage s of this warp: 16 keys of K then of V in 16-byte chunks, rows past kw1 zero-filled;
+    // one commit for every stage number (empty past the last) keeps the group count uniform
+    auto issue = [&](int s) {
+        if (s < nst) {
+            uint8_t* buf = ring + (s % DEC_STAGES) * DEC_STAGE_BYTES;
+#pragma unroll 4
+            for (int i = lane; i < 2 * DEC_SKEYS * 16; i += 32) {
+                const int kv = i >> 8, row = (i >> 4) & 15, c16 = i & 15;
+                const int64_t key = kw0 + (int64_t)s * DEC_SKEYS + row;
+                const bool ok = key < kw1;
+                const uint16_t* src =
+                    (kv ? p.v : p.k) + (ok ? (((int64_t)b * p.Lmax + key) * p.Hkv + hk) * MOBA_D + c16 * 8 : 0);
+                cp_async_16_zfill(smem_u32(buf + kv * DEC_SKEYS * DEC_ROW + row * DEC_ROW + c16 * 16), src, ok);
+            }
+        }
+        dec_commit();
+    };
+    issue(0);
+    issue(1);
+    float o[16][4];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+    float mu0 = -INFINITY, mu1 = -INFINITY;  // running maxima (log2 units) of rows g8, g8 + 8
+    float l0 = 0.f, l1 = 0.f;                // this thread's share of the rows' sums
+    const int mat = lane >> 3, r8 = lane & 7;
+    for (int s = 0; s < nst; ++s) {
+        issue(s + 2);
+        dec_wait_group<2>();  // stage s has landed (the two newer groups may still be in flight)
+        __syncwarp();
+        const uint8_t* kt = ring + (s % DEC_STAGES) * DEC_STAGE_BYTES;
+        const uint8_t* vt = kt + DEC_SKEYS * DEC_ROW;
+        // S = Q K^T for 16 keys: n-tiles of keys 0-7 and 8-15. ldmatrix matrix `mat` of a step:
+        // keys (mat / 2) * 8 .. +7, features ks * 16 + (mat % 2) * 8 .. +7
+        float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         {
-            const int kk = threadIdx.x % DEC_TILE;
-            for (int g = threadIdx.x / DEC_TILE; g < G; g += DEC_THREADS / DEC_TILE) {
-                float s = -INFINITY;
-                if (kk < nk && ((mask >> g) & 1u)) {
-                    float acc = 0.f;
-#pragma unroll 16
-                    for (int e = 0; e < MOBA_D; e += 2) {
-                        const uint32_t w = *reinterpret_cast<const uint32_t*>(&sk[kk][e]);
-                        acc = fmaf(sq[g][e], bf16lo(w), acc);
-                        acc = fmaf(sq[g][e + 1], bf16hi(w), acc);
-                    }
-                    s = acc * p.scale_log2;
-                }
-                sp[g][kk] = s;
+            const uint32_t a0 = smem_u32(kt + ((mat >> 1) * 8 + r8) * DEC_ROW + (mat & 1) * 16);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t b00, b01, b10, b11;
+                dec_ldsm_x4(a0 + ks * 32, b00, b01, b10, b11);
+                dec_mma(sa[0], qa[ks], b00, b01);
+                dec_mma(sa[1], qa[ks], b10, b11);
             }
         }
-        __syncthreads();
-        // online softmax per head: warp w handles heads w, w + 4, ...
-        for (int g = warp; g < G; g += DEC_THREADS / 32) {
-            if (!((mask >> g) & 1u)) continue;
-            const float s0 = sp[g][lane], s1 = sp[g][lane + 32];
-            float mx = fmaxf(s0, s1);
+        // scores in log2 units; keys past the warp's range masked
+        const int64_t key0 = kw0 + (int64_t)s * DEC_SKEYS + 2 * t4;
+        float x[2][4];
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            const float m_old = sm[g];
-            const float m_new = fmaxf(m_old, mx);  // finite: every tile holds at least one key
-            const float p0 = exp2f(s0 - m_new), p1 = exp2f(s1 - m_new);
-            float sum = p0 + p1;
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-            sp[g][lane] = p0;
-            sp[g][lane + 32] = p1;
-            __syncwarp();
-            if (lane == 0) {
-                const float a = exp2f(m_old - m_new);  // 0 on the first tile (m_old = -inf)
-                sa[g] = a;
-                sl[g] = sl[g] * a + sum;
-                sm[g] = m_new;
+            for (int z = 0; z < 4; ++z) {
+                const bool in = key0 + nt * 8 + (z & 1) < kw1;
+                x[nt][z] = in ? sa[nt][z] * p.scale_log2 : -INFINITY;
+            }
+        float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+        float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        // the running maximum moves only when the row maximum passes it by more than 2^8 (so P <= 2^8
+        // stays exact in range); the first stage sets it (its key 0 is a real key)
+        if (mx0 > mu0 + 8.f) {
+            const float f = exp2f(mu0 - mx0);  // 0 on the first stage
+            l0 *= f;
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                o[nt][0] *= f;
+                o[nt][1] *= f;
+            }
+            mu0 = mx0;
+        }
+        if (mx1 > mu1 + 8.f) {
+            const float f = exp2f(mu1 - mx1);
+            l1 *= f;
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                o[nt][2] *= f;
+                o[nt][3] *= f;
+            }
+            mu1 = mx1;
+        }
+        float pr[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            pr[nt][0] = exp2f(x[nt][0] - mu0);
+            pr[nt][1] = exp2f(x[nt][1] - mu0);
+            pr[nt][2] = exp2f(x[nt][2] - mu1);
+            pr[nt][3] = exp2f(x[nt][3] - mu1);
+        }
+        l0 += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+        l1 += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+        // P as the A fragment of O += P V (its 16 keys are the reduction). ldmatrix.trans matrix
+        // `mat` of a step: keys (mat % 2) * 8 .. +7, features np * 16 + (mat / 2) * 8 .. +7
+        const uint32_t pa[4] = {pack_bf16x2(pr[0][0], pr[0][1]), pack_bf16x2(pr[0][2], pr[0][3]),
+                                pack_bf16x2(pr[1][0], pr[1][1]), pack_bf16x2(pr[1][2], pr[1][3])};
+        {
+            const uint32_t a0 = smem_u32(vt + ((mat & 1) * 8 + r8) * DEC_ROW + (mat >> 1) * 16);
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t v0, v1, v2, v3;
+                dec_ldsm_x4_t(a0 + np * 32, v0, v1, v2, v3);
+                dec_mma(o[2 * np], pa, v0, v1);
+                dec_mma(o[2 * np + 1], pa, v2, v3);
             }
         }
-        __syncthreads();
-        // outputs: thread e accumulates feature e of every head that kept the block
-        const int e = threadIdx.x;
+        __syncwarp();  // every lane has read the stage before a later issue refills it
+    }
+    dec_wait_group<0>();
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    // combine the warps: m, l and O of every row through shared memory (over the rings)
+    __syncthreads();
+    float* cm = (float*)smem;                  // [DEC_WARPS][16]
+    float* cl = cm + DEC_WARPS * 16;           // [DEC_WARPS][16]
+    float* co = cl + DEC_WARPS * 16;           // [DEC_WARPS][16][128]
+    if (t4 == 0) {
+        cm[warp * 16 + g8] = nst > 0 ? mu0 : -INFINITY;
+        cm[warp * 16 + g8 + 8] = nst > 0 ? mu1 : -INFINITY;
+        cl[warp * 16 + g8] = l0;
+        cl[warp * 16 + g8 + 8] = l1;
+    }
 #pragma unroll
-        for (int g = 0; g < GM; ++g) {
-            if (!((mask >> g) & 1u)) continue;  // also every g >= G
-            float acc = o[g] * sa[g];
-            for (int kk = 0; kk < nk; ++kk) acc = fmaf(sp[g][kk], bf16_bits_to_float(sv[kk][e]), acc);
-            o[g] = acc;
-        }
+    for (int nt = 0; nt < 16; ++nt) {
+        *reinterpret_cast<float2*>(co + (warp * 16 + g8) * MOBA_D + nt * 8 + 2 * t4) = make_float2(o[nt][0], o[nt][1]);
+        *reinterpret_cast<float2*>(co + (warp * 16 + g8 + 8) * MOBA_D + nt * 8 + 2 * t4) =
+            make_float2(o[nt][2], o[nt][3]);
     }
     __syncthreads();
-    // partial per head that kept the block (an empty chunk writes l = 0)
+    const int e = threadIdx.x;  // output feature
+    for (int g = 0; g < G; ++g) {
+        if (!((mask >> g) & 1u)) continue;
+        float M = -INFINITY;
 #pragma unroll
-    for (int g = 0; g < GM; ++g) {
-        if (!((mask >> g) & 1u)) continue;  // also every g >= G
-        float* pr = p.part + (((bh * p.umax + u) * p.nch + ch) * G + g) * DEC_PART;
-        const bool empty = k1 <= k0;
-        if (threadIdx.x == 0) {
-            pr[0] = empty ? -INFINITY : sm[g];
-            pr[1] = empty ? 0.f : sl[g];
+        for (int w = 0; w < DEC_WARPS; ++w) M = fmaxf(M, cm[w * 16 + g]);
+        float acc = 0.f, ls = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < DEC_WARPS; ++w) {
+                const float f = exp2f(cm[w * 16 + g] - M);  // 0 for a warp without keys
+                acc = fmaf(f, co[(w * 16 + g) * MOBA_D + e], acc);
+                ls = fmaf(f, cl[w * 16 + g], ls);
+            }
         }
-        pr[2 + threadIdx.x] = empty ? 0.f : o[g];
+        float* pr = p.part + (((bh * p.umax + u) * p.nch + ch) * G + g) * DEC_PART;
+        if (e == 0) {
+            pr[0] = M;
+            pr[1] = ls;  // 0 for an empty chunk
+        }
+        pr[4 + e] = acc;
     }
 }
 
 // ---------------------------------------------------------------- merge
 // grid (Hq, B): out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i over the head's partials.
-__global__ void __launch_bounds__(DEC_THREADS) moba_decode_merge_kernel(const DecodeParams p) {
+// Pass 1: the threads stride over the partials for M. Pass 2: warp w takes partials w, w + 8,
+// ... (lane: features 4 lane .. 4 lane + 3); the warps' sums meet in shared memory.
+__global__ void __launch_bounds__(DEC_MERGE_THREADS) moba_decode_merge_kernel(const DecodeParams p) {
+    constexpr int NW = DEC_MERGE_THREADS / 32;
+    __shared__ float red[NW];
+    __shared__ float4 acc_s[NW][32];
+    __shared__ float ls_s[NW];
     const int hq = blockIdx.x, b = blockIdx.y;
     const int hk = hq / p.G, g = hq % p.G;
     const int64_t bh = (int64_t)b * p.Hkv + hk;
-    const int n = p.ucount[bh];
+    const int64_t total = (int64_t)p.ucount[bh] * p.nch;  // partial i: union entry i / nch, chunk i % nch
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float* base = p.part + bh * p.umax * p.nch * (int64_t)p.G * DEC_PART + (int64_t)g * DEC_PART;
+    const uint32_t* um = p.umask + bh * p.umax;
     float M = -INFINITY;
-    for (int u = 0; u < n; ++u) {
-        if (!((p.umask[bh * p.umax + u] >> g) & 1u)) continue;
-        for (int64_t ch = 0; ch < p.nch; ++ch) {
-            const float* pr = p.part + (((bh * p.umax + u) * p.nch + ch) * p.G + g) * DEC_PART;
+    for (int64_t i = threadIdx.x; i < total; i += DEC_MERGE_THREADS)
+        if ((um[i / p.nch] >> g) & 1u) {
+            const float* pr = base + i * p.G * DEC_PART;
             if (pr[1] > 0.f) M = fmaxf(M, pr[0]);
         }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, red[w]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float ls = 0.f;
+#pragma unroll 2
+    for (int64_t i = warp; i < total; i += NW) {
+        if (!((um[i / p.nch] >> g) & 1u)) continue;
+        const float* pr = base + i * p.G * DEC_PART;
+        const float l = pr[1];
+        if (!(l > 0.f)) continue;
+        const float w = exp2f(pr[0] - M);
+        const float4 ov = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
+        acc.x = fmaf(w, ov.x, acc.x);
+        acc.y = fmaf(w, ov.y, acc.y);
+        acc.z = fmaf(w, ov.z, acc.z);
+        acc.w = fmaf(w, ov.w, acc.w);
+        ls = fmaf(w, l, ls);
     }
-    float acc = 0.f, lsum = 0.f;
-    const int e = threadIdx.x;
-    for (int u = 0; u < n; ++u) {
-        if (!((p.umask[bh * p.umax + u] >> g) & 1u)) continue;
-        for (int64_t ch = 0; ch < p.nch; ++ch) {
-            const float* pr = p.part + (((bh * p.umax + u) * p.nch + ch) * p.G + g) * DEC_PART;
-            if (!(pr[1] > 0.f)) continue;
-            const float w = exp2f(pr[0] - M);
-            lsum = fmaf(w, pr[1], lsum);
-            acc = fmaf(w, pr[2 + e], acc);
+    acc_s[warp][lane] = acc;
+    if (lane == 0) ls_s[warp] = ls;
+    __syncthreads();
+    if (threadIdx.x < MOBA_D) {
+        const int e = threadIdx.x;
+        float a = 0.f, lt = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float4 v = acc_s[w][e >> 2];
+            a += (e & 3) == 0 ? v.x : (e & 3) == 1 ? v.y : (e & 3) == 2 ? v.z : v.w;
+            lt += ls_s[w];
         }
+        p.out[((int64_t)b * p.Hq + hq) * MOBA_D + e] = __bfloat16_as_ushort(__float2bfloat16_rn(a / lt));
+        if (e == 0) p.lse[(int64_t)b * p.Hq + hq] = (M + __log2f(lt)) * 0.69314718055994530942f;
     }
-    const float inv = 1.f / lsum;
-    p.out[((int64_t)b * p.Hq + hq) * MOBA_D + e] = __bfloat16_as_ushort(__float2bfloat16_rn(acc * inv));
-    if (e == 0) p.lse[(int64_t)b * p.Hq + hq] = (M + __log2f(lsum)) * 0.69314718055994530942f;
 }

@@ -975,7 +975,7 @@ namespace {
 
 struct DecodePlan {
     int64_t c, umax, nch, nfull_needed;
-    size_t off_count, off_list, off_mask, off_part, total;
+    size_t off_kept, off_count, off_list, off_mask, off_part, total;
 };
 
 int make_decode_plan(int B, int Hq, int Hkv, int64_t L, int d, int bs, int topk, int full, DecodePlan* dp) {
@@ -991,6 +991,8 @@ int make_decode_plan(int B, int Hq, int Hkv, int64_t L, int d, int bs, int topk,
     dp->nch = cdiv(bs, DEC_CHUNK);
     const int64_t units = (int64_t)B * Hkv;
     size_t o = 0;
+    dp->off_kept = o;
+    o = align256(o + sizeof(int32_t) * (size_t)(units * G * (kp > 0 ? kp : 1)));
     dp->off_count = o;
     o = align256(o + sizeof(int32_t) * (size_t)units);
     dp->off_list = o;
@@ -1003,11 +1005,6 @@ int make_decode_plan(int B, int Hq, int Hkv, int64_t L, int d, int bs, int topk,
     return MOBA_OK;
 }
 
-template <int G>
-void launch_decode_attend(const DecodeParams& p, cudaStream_t st) {
-    dim3 grid((unsigned)(p.umax * p.nch), p.Hkv, p.B);
-    moba_decode_attend_kernel<G><<<grid, DEC_THREADS, 0, st>>>(p);
-}
 
 }  // namespace
 
@@ -1088,6 +1085,7 @@ extern "C" int moba_decode(const void* q, const void* k, const void* v, const do
     p.umax = dp.umax;
     p.nch = dp.nch;
     p.full = full_attention;
+    p.kept = (int32_t*)(ws + dp.off_kept);
     p.ucount = (int32_t*)(ws + dp.off_count);
     p.ulist = (int32_t*)(ws + dp.off_list);
     p.umask = (uint32_t*)(ws + dp.off_mask);
@@ -1097,28 +1095,48 @@ extern "C" int moba_decode(const void* q, const void* k, const void* v, const do
     p.lse = lse;
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
     do {
-        const size_t smem_sel = sizeof(double) * (size_t)(dp.c > 0 ? dp.c : 1) +
-                                sizeof(int32_t) * (size_t)p.G * (size_t)(topk > 1 ? topk - 1 : 1);
-        cudaError_t e = cudaFuncSetAttribute(moba_decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem_sel);
-        if (e != cudaSuccess) {
-            rc = cuda_fail(e);
-            break;
+        const int kp = topk - 1;
+        if (!full_attention && dp.c > kp && kp > 0) {  // otherwise no scores are needed
+            const size_t smem_sel = sizeof(double) * (size_t)(dp.c + 8 * kp) + sizeof(int32_t) * (size_t)(8 * kp);
+            cudaError_t e = cudaFuncSetAttribute(moba_decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem_sel);
+            if (e != cudaSuccess) {
+                rc = cuda_fail(e);
+                break;
+            }
+            moba_decode_select_kernel<<<dim3(p.G, Hkv, B), DEC_SEL_THREADS, smem_sel, st>>>(p);
+        } else if (!full_attention) {
+            moba_decode_select_kernel<<<dim3(p.G, Hkv, B), DEC_SEL_THREADS, 0, st>>>(p);
         }
-        moba_decode_select_kernel<<<dim3(Hkv, B), DEC_THREADS, full_attention ? 0 : smem_sel, st>>>(p);
-        count_launch();
-        if ((rc = launch_ok())) break;
-        switch (p.G) {
-            case 1: launch_decode_attend<1>(p, st); break;
-            case 2: launch_decode_attend<2>(p, st); break;
-            case 3: launch_decode_attend<3>(p, st); break;
-            case 4: launch_decode_attend<4>(p, st); break;
-            case 5: case 6: case 7: case 8: launch_decode_attend<8>(p, st); break;
-            default: launch_decode_attend<16>(p, st); break;  // 9 .. 16 (make_decode_plan caps G)
+        if (!full_attention) {
+            count_launch();
+            if ((rc = launch_ok())) break;
         }
-        count_launch();
-        if ((rc = launch_ok())) break;
-        moba_decode_merge_kernel<<<dim3(Hq, B), DEC_THREADS, 0, st>>>(p);
+        {
+            const size_t smem_union = full_attention ? 0 : sizeof(uint32_t) * (size_t)(dp.c > 0 ? dp.c : 1);
+            cudaError_t e = cudaFuncSetAttribute(moba_decode_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem_union);
+            if (e != cudaSuccess) {
+                rc = cuda_fail(e);
+                break;
+            }
+            moba_decode_union_kernel<<<dim3(Hkv, B), DEC_UNION_THREADS, smem_union, st>>>(p);
+            count_launch();
+            if ((rc = launch_ok())) break;
+        }
+        {
+            cudaError_t e = cudaFuncSetAttribute(moba_decode_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 DEC_ATTEND_SMEM);
+            if (e != cudaSuccess) {
+                rc = cuda_fail(e);
+                break;
+            }
+            dim3 grid((unsigned)(p.umax * p.nch), Hkv, B);
+            moba_decode_attend_kernel<<<grid, DEC_WARPS * 32, DEC_ATTEND_SMEM, st>>>(p);
+            count_launch();
+            if ((rc = launch_ok())) break;
+        }
+        moba_decode_merge_kernel<<<dim3(Hq, B), DEC_MERGE_THREADS, 0, st>>>(p);
         count_launch();
         rc = launch_ok();
     } while (0);
