@@ -11,15 +11,15 @@
 //
 // Four kernels:
 //   select  one CTA per query head: exact fp64 scores against the cached block
-//           summaries Kbar into shared memory; each warp picks the best topk - 1
-//           of a quarter of the blocks by rounds of a warp arg-max over per-lane
-//           maxima (only the lane that lost its maximum rescans), and warp 0 picks
-//           the head's topk - 1 among the four lists the same way;
+//           summaries Kbar into shared memory (a warp per summary row, coalesced);
+//           each warp keeps the best topk - 1 of a slice of the blocks by counting,
+//           for each block, the blocks of the slice that rank before it; the head's
+//           topk - 1 are the warps' winners of rank < topk - 1 among all of them;
 //   union   one CTA per (b, kv head): the union of the group's kept blocks in
 //           ascending order with a G-bit mask per block (the heads that kept it),
 //           so each K/V block is read once for the whole group;
-//   attend  one CTA per (b, kv head, union entry, 512-key chunk), four warps of
-//           128 keys each. A warp streams its keys and values through its own
+//   attend  one CTA per (b, kv head, union entry, chunk of 512 to 4096 keys), four
+//           warps of a quarter chunk each. A warp streams its keys and values through its own
 //           3-stage cp.async ring of 16-key stages and runs both products on the
 //           tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate) with the
 //           group's heads as the 16 rows: S = Q K^T, an online softmax per row,
@@ -32,11 +32,11 @@
 #include "common.cuh"
 
 #define DEC_MAX_G 16        // query heads per kv head: the 16 rows of an m16n8k16 product
-#define DEC_SEL_THREADS 128
+#define DEC_SEL_THREADS 512
+#define DEC_SEL_WARPS (DEC_SEL_THREADS / 32)
 #define DEC_UNION_THREADS 256
 #define DEC_WARPS 4
-#define DEC_CHUNK 512                               // keys per attend CTA
-#define DEC_WARP_KEYS (DEC_CHUNK / DEC_WARPS)       // keys per warp
+#define DEC_MIN_CHUNK 512                           // keys per attend CTA, at least (the host may double it)
 #define DEC_SKEYS 16                                // keys per ring stage
 #define DEC_STAGES 3
 #define DEC_ROW 272  // bytes per staged key row: 256 + 16, so the 8 rows one ldmatrix reads hit distinct banks
@@ -58,6 +58,7 @@ struct DecodeParams {
     int B, Hq, Hkv, G, bs, topk;
     int64_t c;            // own block of the query
     int64_t umax;         // union capacity per (b, kv head)
+    int64_t chunk;        // keys per attend CTA (a multiple of DEC_WARPS * DEC_SKEYS)
     int64_t nch;          // chunks per block
     int full;             // keep every block
     int32_t* kept;        // [B*Hkv][G][max(topk - 1, 1)] kept earlier blocks per head, ascending
@@ -71,75 +72,27 @@ struct DecodeParams {
     float scale_log2;     // log2(e) / sqrt(d)
 };
 
-// (score desc, block asc): does (s2, j2) rank before (s, j)? A NaN score never ranks first.
+// (score desc, block asc): does (s2, j2) rank before (s, j)?
 __device__ __forceinline__ bool dec_before(double s2, int32_t j2, double s, int32_t j) {
     return s2 > s || (s2 == s && j2 < j);
 }
 
-// Warp arg-max of (s, j) by dec_before; every lane gets the winner.
-__device__ __forceinline__ void dec_warp_best(double& s, int32_t& j) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const double s2 = __shfl_xor_sync(0xffffffffu, s, o);
-        const int32_t j2 = __shfl_xor_sync(0xffffffffu, j, o);
-        if (dec_before(s2, j2, s, j)) {
-            s = s2;
-            j = j2;
-        }
-    }
-}
-
-// Rounds of a warp arg-max over the n scores sc[0 .. n) with block ids jd[i] (i itself when jd
-// is null): lane l owns entries l, l + 32, ...; each round's winner is struck out (set to NaN,
-// which never ranks first) and only its owner rescans. Lane 0 writes up to `want` winners in
-// rank order to ws / wj; returns their number (the same on every lane).
-__device__ __forceinline__ int dec_rounds(double* sc, const int32_t* jd, int n, int want, double* ws, int32_t* wj,
-                                          int lane) {
-    double lb = -INFINITY;
-    int32_t lj = 0x7FFFFFFF;
-    int li = -1;
-    auto rescan = [&]() {
-        lb = -INFINITY;
-        lj = 0x7FFFFFFF;
-        li = -1;
-        for (int i = lane; i < n; i += 32) {
-            const double s = sc[i];
-            const int32_t j = jd ? jd[i] : i;
-            if (dec_before(s, j, lb, lj)) {
-                lb = s;
-                lj = j;
-                li = i;
-            }
-        }
-    };
-    rescan();
-    int got = 0;
-    for (; got < want; ++got) {
-        double bs = lb;
-        int32_t bj = lj;
-        dec_warp_best(bs, bj);
-        if (bj == 0x7FFFFFFF) break;  // nothing left
-        if (lane == 0) {
-            ws[got] = bs;
-            wj[got] = bj;
-        }
-        if (li >= 0 && lj == bj) {  // this lane owned the winner
-            sc[li] = __longlong_as_double(0x7FF8000000000000ll);
-            rescan();
-        }
-        __syncwarp();
-    }
-    return got;
+// Rank of entry i among the n entries (sc[k], jd[k]) by dec_before: how many rank before it.
+// The ranks of distinct blocks are distinct, so the entries of rank < m are the m best.
+// Lanes of a warp that scan the same array read each entry at the same time (a broadcast).
+__device__ __forceinline__ int dec_rank(const double* sc, const int32_t* jd, int n, double s, int32_t j) {
+    int rank = 0;
+    for (int k = 0; k < n; ++k) rank += dec_before(sc[k], jd[k], s, j);
+    return rank;
 }
 
 // ---------------------------------------------------------------- select
-// grid (G, Hkv, B); dynamic smem (when c > topk - 1 > 0): the c scores, then two areas of 4 (topk - 1)
-// (score, block) candidates: the four warps' lists and their compacted merge.
+// grid (G, Hkv, B); dynamic smem (when c > topk - 1 > 0): the c scores, two areas of
+// DEC_SEL_WARPS (topk - 1) (score, block) candidates (the warps' lists and their compacted
+// merge), then the c block ids.
 __global__ void __launch_bounds__(DEC_SEL_THREADS) moba_decode_select_kernel(const DecodeParams p) {
     extern __shared__ __align__(16) uint8_t smem[];
-    __shared__ double sq[MOBA_D];
-    __shared__ int32_t cnt[DEC_SEL_THREADS / 32];
-    __shared__ double fs[MOBA_MAX_TOPK];
+    __shared__ int32_t cnt[DEC_SEL_WARPS];
     __shared__ int32_t fj[MOBA_MAX_TOPK];
     const int g = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
     const int hq = hk * p.G + g;
@@ -150,51 +103,77 @@ __global__ void __launch_bounds__(DEC_SEL_THREADS) moba_decode_select_kernel(con
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int32_t* kept = p.kept + (bh * p.G + g) * (kp > 0 ? kp : 1);
     if (c > kp && kp > 0) {
+        constexpr int NW = DEC_SEL_WARPS;
         double* sc = (double*)smem;                  // [c] scores
-        double* cs = sc + c;                         // [4][kp] candidate scores per warp
-        double* ms = cs + 4 * kp;                    // [4 kp] the compacted candidates
-        int32_t* cj = (int32_t*)(ms + 4 * kp);       // [4][kp] candidate blocks per warp
-        int32_t* mj = cj + 4 * kp;                   // [4 kp]
-        const uint16_t* qr = p.q + ((int64_t)b * p.Hq + hq) * MOBA_D;
-        for (int e = threadIdx.x; e < MOBA_D; e += DEC_SEL_THREADS) sq[e] = (double)bf16_bits_to_float(qr[e]);
-        __syncthreads();
-        // exact fp64 scores <q, Kbar_j>, features ascending (one fused multiply-add each); a NaN
-        // score ranks as -inf
-        for (int64_t j = threadIdx.x; j < c; j += DEC_SEL_THREADS) {
-            const double* kb = p.kbar + (bh * p.kbar_rows + j) * MOBA_D;
-            double s = 0.0;
-#pragma unroll 8
-            for (int e = 0; e < MOBA_D; ++e) s = fma(sq[e], kb[e], s);
-            sc[j] = (s == s) ? s : -INFINITY;
-        }
-        __syncthreads();
-        // each warp: the best kp of its quarter of the blocks
-        const int lo = (int)(c * warp / 4), hi = (int)(c * (warp + 1) / 4);
-        const int n = dec_rounds(sc + lo, nullptr, hi - lo, kp, cs + warp * kp, cj + warp * kp, lane);
-        __syncwarp();
-        if (lane == 0) {
-            for (int i = 0; i < n; ++i) cj[warp * kp + i] += lo;  // block ids
-            cnt[warp] = n;
-        }
-        __syncthreads();
-        if (warp == 0) {  // the head's best kp among the four lists, by the same rounds
-            int off = 0;
-            for (int w = 0; w < 4; ++w) {
-                for (int i = lane; i < cnt[w]; i += 32) {
-                    ms[off + i] = cs[w * kp + i];
-                    mj[off + i] = cj[w * kp + i];
+        double* cs = sc + c;                         // [NW][kp] candidate scores per warp
+        double* ms = cs + NW * kp;                   // [NW kp] the compacted candidates
+        int32_t* cj = (int32_t*)(ms + NW * kp);      // [NW][kp] candidate blocks per warp
+        int32_t* mj = cj + NW * kp;                  // [NW kp]
+        int32_t* sj = mj + NW * kp;                  // [c] block ids
+        // exact fp64 scores <q, Kbar_j>: a warp per row, lane l multiplies features 4l .. 4l + 3
+        // (fused multiply-adds in feature order), then a butterfly sum over the lanes. Eight rows
+        // per warp are in flight at once. A NaN score ranks as -inf.
+        constexpr int RW = 8;
+        const uint16_t* qr = p.q + ((int64_t)b * p.Hq + hq) * MOBA_D + 4 * lane;
+        const uint2 qw = *reinterpret_cast<const uint2*>(qr);
+        const double q0 = bf16lo(qw.x), q1 = bf16hi(qw.x), q2 = bf16lo(qw.y), q3 = bf16hi(qw.y);
+        const double* kb0 = p.kbar + bh * p.kbar_rows * MOBA_D + 4 * lane;
+        for (int64_t j0 = warp; j0 < c; j0 += RW * NW) {
+            double2 a[RW], bq[RW];
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                const int64_t j = j0 + (int64_t)r * NW;
+                a[r] = make_double2(0.0, 0.0);
+                bq[r] = a[r];
+                if (j < c) {
+                    a[r] = *reinterpret_cast<const double2*>(kb0 + j * MOBA_D);
+                    bq[r] = *reinterpret_cast<const double2*>(kb0 + j * MOBA_D + 2);
                 }
-                off += cnt[w];
             }
-            __syncwarp();
-            const int m = dec_rounds(ms, mj, off, kp, fs, fj, lane);
-            __syncwarp();
-            // ascending block order: winner i goes to its rank among the m winners
-            for (int i = lane; i < m; i += 32) {
-                int rank = 0;
-                for (int t = 0; t < m; ++t) rank += fj[t] < fj[i];
-                kept[rank] = fj[i];
+#pragma unroll
+            for (int r = 0; r < RW; ++r) {
+                double part = fma(q3, bq[r].y, fma(q2, bq[r].x, fma(q1, a[r].y, q0 * a[r].x)));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+                const int64_t j = j0 + (int64_t)r * NW;
+                if (lane == 0 && j < c) sc[j] = (part == part) ? part : -INFINITY;
             }
+        }
+        __syncthreads();
+        // block ids of the scores, for the rank counts
+        for (int64_t j = threadIdx.x; j < c; j += DEC_SEL_THREADS) sj[j] = (int32_t)j;
+        __syncthreads();
+        // each warp: the best kp of its slice of the blocks, by rank counts within the slice
+        const int lo = (int)(c * warp / NW), hi = (int)(c * (warp + 1) / NW);
+        for (int i = lo + lane; i < hi; i += 32) {
+            const int rank = dec_rank(sc + lo, sj + lo, hi - lo, sc[i], i);
+            if (rank < kp) {
+                cs[warp * kp + rank] = sc[i];
+                cj[warp * kp + rank] = i;
+            }
+        }
+        if (lane == 0) cnt[warp] = (hi - lo < kp) ? hi - lo : kp;
+        __syncthreads();
+        // the head's best kp among the warps' lists, by rank counts over the compacted lists
+        int n = 0;
+        for (int w = 0; w < NW; ++w) {
+            for (int i = threadIdx.x; i < cnt[w]; i += DEC_SEL_THREADS) {
+                ms[n + i] = cs[w * kp + i];
+                mj[n + i] = cj[w * kp + i];
+            }
+            n += cnt[w];
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += DEC_SEL_THREADS) {
+            const int rank = dec_rank(ms, mj, n, ms[i], mj[i]);
+            if (rank < kp) fj[rank] = mj[i];
+        }
+        __syncthreads();
+        // ascending block order: winner i goes to its rank among the kp winners
+        for (int i = threadIdx.x; i < kp; i += DEC_SEL_THREADS) {
+            int pos = 0;
+            for (int t = 0; t < kp; ++t) pos += fj[t] < fj[i];
+            kept[pos] = fj[i];
         }
     } else {
         for (int j = threadIdx.x; j < npast; j += DEC_SEL_THREADS) kept[j] = j;  // every earlier block
@@ -305,14 +284,15 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 2) moba_decode_attend_kernel(c
     const int64_t j = p.ulist[bh * p.umax + u];
     const uint32_t mask = p.umask[bh * p.umax + u];
     const int64_t bend = (j == p.c) ? p.L : (j + 1) * p.bs;  // keys [j*bs, bend)
-    const int64_t k0 = j * p.bs + ch * DEC_CHUNK;
-    const int64_t k1 = (k0 + DEC_CHUNK < bend) ? k0 + DEC_CHUNK : bend;
+    const int64_t k0 = j * p.bs + ch * p.chunk;
+    const int64_t k1 = (k0 + p.chunk < bend) ? k0 + p.chunk : bend;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g8 = lane >> 2, t4 = lane & 3;
     const int G = p.G;
-    // this warp's keys [kw0, kw1), in stages of 16
-    const int64_t kw0 = k0 + warp * DEC_WARP_KEYS;
-    const int64_t kw1 = (kw0 + DEC_WARP_KEYS < k1) ? kw0 + DEC_WARP_KEYS : (k1 > kw0 ? k1 : kw0);
+    // this warp's keys [kw0, kw1): a quarter of the chunk, in stages of 16
+    const int64_t wk = p.chunk / DEC_WARPS;
+    const int64_t kw0 = k0 + warp * wk;
+    const int64_t kw1 = (kw0 + wk < k1) ? kw0 + wk : (k1 > kw0 ? k1 : kw0);
     const int nst = (int)((kw1 - kw0 + DEC_SKEYS - 1) / DEC_SKEYS);
 
     // Q as A fragments, 8 steps of 16 features
@@ -487,7 +467,8 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 2) moba_decode_attend_kernel(c
 // ---------------------------------------------------------------- merge
 // grid (Hq, B): out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i over the head's partials.
 // Pass 1: the threads stride over the partials for M. Pass 2: warp w takes partials w, w + 8,
-// ... (lane: features 4 lane .. 4 lane + 3); the warps' sums meet in shared memory.
+// ... (lane: features 4 lane .. 4 lane + 3); the warps' sums meet in shared memory. Both passes
+// issue four partials' loads before using any.
 __global__ void __launch_bounds__(DEC_MERGE_THREADS) moba_decode_merge_kernel(const DecodeParams p) {
     constexpr int NW = DEC_MERGE_THREADS / 32;
     __shared__ float red[NW];
@@ -501,11 +482,23 @@ __global__ void __launch_bounds__(DEC_MERGE_THREADS) moba_decode_merge_kernel(co
     const float* base = p.part + bh * p.umax * p.nch * (int64_t)p.G * DEC_PART + (int64_t)g * DEC_PART;
     const uint32_t* um = p.umask + bh * p.umax;
     float M = -INFINITY;
-    for (int64_t i = threadIdx.x; i < total; i += DEC_MERGE_THREADS)
-        if ((um[i / p.nch] >> g) & 1u) {
-            const float* pr = base + i * p.G * DEC_PART;
-            if (pr[1] > 0.f) M = fmaxf(M, pr[0]);
+    for (int64_t i0 = threadIdx.x; i0 < total; i0 += 4 * DEC_MERGE_THREADS) {
+        float mv[4], lv[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int64_t i = i0 + (int64_t)r * DEC_MERGE_THREADS;
+            lv[r] = 0.f;
+            mv[r] = -INFINITY;
+            if (i < total && ((um[i / p.nch] >> g) & 1u)) {
+                const float* pr = base + i * p.G * DEC_PART;
+                mv[r] = pr[0];
+                lv[r] = pr[1];
+            }
         }
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            if (lv[r] > 0.f) M = fmaxf(M, mv[r]);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     if (lane == 0) red[warp] = M;
@@ -515,19 +508,33 @@ __global__ void __launch_bounds__(DEC_MERGE_THREADS) moba_decode_merge_kernel(co
     for (int w = 0; w < NW; ++w) M = fmaxf(M, red[w]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float ls = 0.f;
-#pragma unroll 2
-    for (int64_t i = warp; i < total; i += NW) {
-        if (!((um[i / p.nch] >> g) & 1u)) continue;
-        const float* pr = base + i * p.G * DEC_PART;
-        const float l = pr[1];
-        if (!(l > 0.f)) continue;
-        const float w = exp2f(pr[0] - M);
-        const float4 ov = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
-        acc.x = fmaf(w, ov.x, acc.x);
-        acc.y = fmaf(w, ov.y, acc.y);
-        acc.z = fmaf(w, ov.z, acc.z);
-        acc.w = fmaf(w, ov.w, acc.w);
-        ls = fmaf(w, l, ls);
+    // four partials per warp and iteration, every load issued before any is used
+    for (int64_t i0 = warp; i0 < total; i0 += 4 * NW) {
+        float mv[4], lv[4];
+        float4 ov[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int64_t i = i0 + (int64_t)r * NW;
+            lv[r] = 0.f;
+            mv[r] = 0.f;
+            ov[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < total && ((um[i / p.nch] >> g) & 1u)) {
+                const float* pr = base + i * p.G * DEC_PART;
+                mv[r] = pr[0];
+                lv[r] = pr[1];
+                ov[r] = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            if (!(lv[r] > 0.f)) continue;
+            const float w = exp2f(mv[r] - M);
+            acc.x = fmaf(w, ov[r].x, acc.x);
+            acc.y = fmaf(w, ov[r].y, acc.y);
+            acc.z = fmaf(w, ov[r].z, acc.z);
+            acc.w = fmaf(w, ov[r].w, acc.w);
+            ls = fmaf(w, lv[r], ls);
+        }
     }
     acc_s[warp][lane] = acc;
     if (lane == 0) ls_s[warp] = ls;

@@ -974,7 +974,7 @@ extern "C" int moba_gate_varlen(const void* q, const void* k, int32_t* idx, cons
 namespace {
 
 struct DecodePlan {
-    int64_t c, umax, nch, nfull_needed;
+    int64_t c, umax, chunk, nch, nfull_needed;
     size_t off_kept, off_count, off_list, off_mask, off_part, total;
 };
 
@@ -988,7 +988,23 @@ int make_decode_plan(int B, int Hq, int Hkv, int64_t L, int d, int bs, int topk,
     const int64_t kp = topk - 1;
     const int64_t past = full ? dp->c : (dp->c < (int64_t)G * kp ? dp->c : (int64_t)G * kp);
     dp->umax = past + 1;
-    dp->nch = cdiv(bs, DEC_CHUNK);
+    // keys per attend CTA: 512, doubled (up to 4096, not past the block) while the grid keeps at
+    // least 8 CTAs per SM, so that long unions run fewer, longer CTAs (each pays its pipeline
+    // fill and combine once) with fewer partials to merge
+    int nsm = 148;
+    {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm < 1) {
+            cudaGetLastError();
+            nsm = 148;
+        }
+    }
+    dp->chunk = DEC_MIN_CHUNK;
+    while (dp->chunk < 4096 && dp->chunk < bs &&
+           (int64_t)B * Hkv * dp->umax * cdiv(bs, 2 * dp->chunk) >= 8 * (int64_t)nsm)
+        dp->chunk *= 2;
+    dp->nch = cdiv(bs, dp->chunk);
     const int64_t units = (int64_t)B * Hkv;
     size_t o = 0;
     dp->off_kept = o;
@@ -1083,6 +1099,7 @@ extern "C" int moba_decode(const void* q, const void* k, const void* v, const do
     p.topk = topk;
     p.c = dp.c;
     p.umax = dp.umax;
+    p.chunk = dp.chunk;
     p.nch = dp.nch;
     p.full = full_attention;
     p.kept = (int32_t*)(ws + dp.off_kept);
@@ -1097,7 +1114,8 @@ extern "C" int moba_decode(const void* q, const void* k, const void* v, const do
     do {
         const int kp = topk - 1;
         if (!full_attention && dp.c > kp && kp > 0) {  // otherwise no scores are needed
-            const size_t smem_sel = sizeof(double) * (size_t)(dp.c + 8 * kp) + sizeof(int32_t) * (size_t)(8 * kp);
+            const size_t smem_sel = sizeof(double) * (size_t)(dp.c + 2 * DEC_SEL_WARPS * kp) +
+                                    sizeof(int32_t) * (size_t)(2 * DEC_SEL_WARPS * kp + dp.c);
             cudaError_t e = cudaFuncSetAttribute(moba_decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)smem_sel);
             if (e != cudaSuccess) {
