@@ -14,8 +14,9 @@
 // (tcgen05, fp32 accumulation; keys on the TMEM lanes):
 //   S^T  = K Q^T          SS (K, Q K-major)                  -> TMEM S
 //   dP^T = V dO^T         SS (V, dO K-major)                 -> TMEM dP
-//   P^T, dS^T  by the 128 threads (thread = key), bf16 into TMEM over S / dP,
-//              dS also into shared memory (the A operand of dQ, query-major)
+//   P^T, dS^T  by the 256 threads (two per key, each half of the queries), bf16
+//              into TMEM over S / dP, dS also into shared memory (the A operand
+//              of dQ, query-major)
 //   dV += P^T dO          TS (A from TMEM, dO MN-major)
 //   dK += dS^T Q          TS (A from TMEM, Q MN-major)
 //   dQ  = dS K            SS (dS MN-major, K MN-major)       -> TMEM S
@@ -24,13 +25,15 @@
 //   the products are done) and adds it with one bulk reduction
 //   (cp.reduce.async.bulk .add.f32), which the L2 performs about three times as
 //   fast as per-thread vector atomics; a last kernel scales and rounds to bf16.
-// Roles are not split: one warpgroup gathers, waits, computes and reduces in turn.
+// Roles are not split: two warpgroups gather, wait, compute and reduce in turn,
+// warps w and w + 4 sharing TMEM lanes 32 (w % 4) .. + 31 (a key, or a query for
+// dQ) and splitting the columns, so each scheduler has two warps to switch between.
 #pragma once
 #include <cuda.h>
 
 #include "k_attn_tc.cuh"
 
-#define BWD_THREADS 128
+#define BWD_THREADS 256
 #define BWD_TILE_BYTES 32768  // 128 rows x 128 d x bf16
 #define BWD_SMEM_BYTES (5 * BWD_TILE_BYTES + 2048 + 1024)
 #define BWD_DQ_STRIDE 528  // bytes per staged dQ row: 512 + 16, so 8 threads storing 16 bytes each hit distinct banks
@@ -136,7 +139,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     int64_t* sRow = (int64_t*)(sD + 128);       // dq_acc row offset of each query row, -1 if empty
     BwdBars* bars = (BwdBars*)(smem_raw + 5 * BWD_TILE_BYTES + 2048);
     const int warp = threadIdx.x >> 5;
-    const int r = threadIdx.x;  // TMEM lane: a key (S^T, dP^T, dK, dV) or a query (dQ)
+    const int r = threadIdx.x & 127;  // TMEM lane: a key (S^T, dP^T, dK, dV) or a query (dQ)
+    const int h = threadIdx.x >> 7;   // which half of the columns this thread takes
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
@@ -154,7 +158,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tS = tmem, tP = tmem + 128, tK = tmem + 256, tV = tmem + 384;
     const uint32_t idesc_ss = make_idesc_bf16(128, 128, 0, 0);   // both K-major
     const uint32_t idesc_ts = make_idesc_bf16(128, 128, 0, 1);   // A in TMEM, B MN-major
@@ -235,14 +239,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                 const uint16_t* srcg = p.dout + (valid ? qrow * MOBA_D : 0);
                 const uint32_t dq_s = smem_u32(sQ) + r * 128, dg_s = smem_u32(sG) + r * 128;
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
+                for (int c = 8 * h; c < 8 * h + 8; ++c) {  // this thread's 64 features
                     const uint32_t off = (c >> 3) * 16384 + (((c & 7) ^ (r & 7)) << 4);
                     cp_async_16_zfill(dq_s + off, srcq + c * 8, valid);
                     cp_async_16_zfill(dg_s + off, srcg + c * 8, valid);
                 }
-                sL[r] = valid ? p.lse[lrow] * 1.4426950408889634f : INFINITY;
-                sD[r] = valid ? p.Dvec[lrow] : 0.f;
-                sRow[r] = valid ? qrow : -1;
+                if (h == 0) {
+                    sL[r] = valid ? p.lse[lrow] * 1.4426950408889634f : INFINITY;
+                    sD[r] = valid ? p.Dvec[lrow] : 0.f;
+                    sRow[r] = valid ? qrow : -1;
+                }
                 cp_async_wait_all();
                 fence_proxy_async_smem();
             }
@@ -268,12 +274,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             if (!(ok = __syncthreads_and(ok))) break;
             ++mma_phase;
             tc_fence_after();
-            // ---- P^T and dS^T for key r, 32 query columns at a time
+            // ---- P^T and dS^T for key r, 32 query columns at a time: this thread's two chunks
+            // qq = 2h, 2h + 1 (queries 64h .. 64h + 63)
             {
                 const int64_t key = u0 + r;
                 const bool key_ok = r < ku;
 #pragma unroll 1
-                for (int qq = 0; qq < 4; ++qq) {
+                for (int qq = 2 * h; qq < 2 * h + 2; ++qq) {
                     uint32_t s32[32], g32[32];
                     tmem_ld32(tS + lane_off + qq * 32, s32);
                     tmem_ld32(tP + lane_off + qq * 32, g32);
@@ -295,10 +302,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                         pk[i / 2] = pack_bf16x2(pv[0], pv[1]);
                         dk2[i / 2] = pack_bf16x2(dsv[0], dsv[1]);
                     }
-                    // P^T over S columns [16 qq, 16 qq + 16) and dS^T over the same dP columns: every
-                    // column up to 32 qq + 31 has been read, so nothing unread is overwritten
-                    tmem_st16(tS + lane_off + qq * 16, pk);
-                    tmem_st16(tP + lane_off + qq * 16, dk2);
+                    // P^T over S columns [64h + 16 (qq - 2h), +16) and dS^T over the same dP columns:
+                    // inside this thread's first chunk [64h, 64h + 32), which it has read, and which
+                    // no other thread reads (queries 16k .. 16k + 15 end up at column 8k + 32 [k >= 4])
+                    tmem_st16(tS + lane_off + 64 * h + 16 * (qq - 2 * h), pk);
+                    tmem_st16(tP + lane_off + 64 * h + 16 * (qq - 2 * h), dk2);
                     // dS into shared memory, query-major: half qq / 2 holds queries 64 (qq / 2) .. +63,
                     // row r (this key) of 128 bytes, 16-byte chunks swizzled by (r & 7)
                     uint8_t* drow = sS + (qq >> 1) * 16384 + r * 128;
@@ -318,12 +326,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             // ---- dV += P^T dO, dK += dS^T Q, dQ = dS K (into S)
             if (threadIdx.x == 0) {
                 const uint32_t first = qt == 0 ? 0u : 1u;  // the item's first tile starts dK, dV
+                // packed P^T / dS^T of queries 16k .. 16k + 15 sit at column 8k (k < 4), 8k + 32 (k >= 4)
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    tc_mma_ts(tV, tS + k * 8, dG_mn + k * 128, idesc_ts, (k > 0 || first) ? 1u : 0u);
+                    tc_mma_ts(tV, tS + k * 8 + (k >= 4 ? 32 : 0), dG_mn + k * 128, idesc_ts, (k > 0 || first) ? 1u : 0u);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    tc_mma_ts(tK, tP + k * 8, dQ_mn + k * 128, idesc_ts, (k > 0 || first) ? 1u : 0u);
+                    tc_mma_ts(tK, tP + k * 8 + (k >= 4 ? 32 : 0), dQ_mn + k * 128, idesc_ts, (k > 0 || first) ? 1u : 0u);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) tc_mma_ss(tS, dS_mn + k * 128, dK_mn + k * 128, idesc_dq, k > 0 ? 1u : 0u);
                 tc_commit(&bars->mma);
@@ -339,7 +348,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                 const int64_t dst = sRow[r];
                 float* stage = (float*)(sQ + r * BWD_DQ_STRIDE);
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 2 * h; c < 2 * h + 2; ++c) {  // this thread's half of the row
                     uint32_t v[32];
                     tmem_ld32(tS + lane_off + c * 32, v);
                     tc_wait_ld();
@@ -349,7 +358,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                 }
                 if (dst >= 0) {
                     fence_proxy_async_smem();  // the staged row is visible to the bulk-copy unit
-                    bulk_reduce_add_f32(p.dq_acc + dst * MOBA_D, smem_u32(stage), MOBA_D * 4);
+                    bulk_reduce_add_f32(p.dq_acc + dst * MOBA_D + 64 * h, smem_u32(stage + 64 * h), MOBA_D * 2);
                     bulk_commit();
                 }
                 bulk_wait_read();  // the row is read before the next tile's gather overwrites it
@@ -365,7 +374,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             const bool key_ok = r < ku;
             const int64_t krow = ((int64_t)b * p.N + u0 + r) * p.Hkv + hk;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * h; c < 2 * h + 2; ++c) {  // this thread's half of the features
                 uint32_t a[32], v[32];
                 tmem_ld32(tK + lane_off + c * 32, a);
                 tmem_ld32(tV + lane_off + c * 32, v);
