@@ -276,7 +276,7 @@ __device__ __forceinline__ void dec_wait_group() {
 // and 2 t4 + 8 (+1); B column g8, rows 2 t4 (+1) and 2 t4 + 8 (+1); C rows g8 and g8 + 8,
 // columns 2 t4 (+1). The rows are the group's heads, zero beyond G.
 __global__ void __launch_bounds__(DEC_WARPS * 32, 2) moba_decode_attend_kernel(const DecodeParams p) {
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(16) uint8_t smem[];  // 16-byte rows for cp.async and ldmatrix
     const int hk = blockIdx.y, b = blockIdx.z;
     const int64_t bh = (int64_t)b * p.Hkv + hk;
     const int64_t u = blockIdx.x / p.nch, ch = blockIdx.x % p.nch;
