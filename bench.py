@@ -718,7 +718,7 @@ def run_decode(args):
         "config": {"workload": "decode step, KV cache of " + workload_name(w), "global_batch": B, "seq_len": L,
                    "parallelism": "single GPU", "l2": "a 256 MB buffer is rewritten before every timed step"},
         "tokens_per_s": B / (m["us"] * 1e-6),
-        "roofline": {"kernel": "moba decode (select + attend + merge)", "bound": "hbm", "achieved": m["achieved_gbs"],
+        "roofline": {"kernel": "moba decode (select, union, attend, merge)", "bound": "hbm", "achieved": m["achieved_gbs"],
                      "peak": hbm, "unit": "GB/s", "frac": m["achieved_gbs"] / hbm, "traffic": None,
                      "bytes_per_step": m["bytes"], "peak_source": f"hbm_gbs of {peak_src}"},
         "full_attention_decode": res["full"],
