@@ -28,8 +28,16 @@
 //   merge   one CTA per (b, query head): log-sum-exp merge of its partials, the
 //           warps splitting the partials.
 // Memory bound: the K/V bytes of the union blocks dominate.
+//
+// union, attend and merge are launched as programmatic dependents of the kernel before them
+// (the launch overlaps that kernel's tail): each waits for its predecessor's results with
+// griddepcontrol.wait before reading them, and attend loads its queries (the caller's input,
+// complete before select started) before it waits. Launched plainly, both instructions do nothing.
 #pragma once
 #include "common.cuh"
+
+__device__ __forceinline__ void dec_wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void dec_allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 #define DEC_MAX_G 16        // query heads per kv head: the 16 rows of an m16n8k16 product
 #define DEC_SEL_THREADS 512
@@ -102,6 +110,7 @@ __global__ void __launch_bounds__(DEC_SEL_THREADS) moba_decode_select_kernel(con
     const int npast = (int)(c < kp ? c : kp);  // earlier blocks kept
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int32_t* kept = p.kept + (bh * p.G + g) * (kp > 0 ? kp : 1);
+    dec_allow_dependents();
     if (c > kp && kp > 0) {
         constexpr int NW = DEC_SEL_WARPS;
         double* sc = (double*)smem;                  // [c] scores
@@ -198,6 +207,8 @@ __global__ void __launch_bounds__(DEC_UNION_THREADS) moba_decode_union_kernel(co
     const uint32_t all = (1u << p.G) - 1u;  // G <= 16
     int32_t* ul = p.ulist + bh * p.umax;
     uint32_t* um = p.umask + bh * p.umax;
+    dec_wait_prior_grid();  // select's kept lists (and the previous step's readers of the union) are done
+    dec_allow_dependents();
     if (p.full) {  // every block 0 .. c, kept by every head
         for (int64_t j = threadIdx.x; j <= c; j += DEC_UNION_THREADS) {
             ul[j] = (int32_t)j;
@@ -280,22 +291,11 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 2) moba_decode_attend_kernel(c
     const int hk = blockIdx.y, b = blockIdx.z;
     const int64_t bh = (int64_t)b * p.Hkv + hk;
     const int64_t u = blockIdx.x / p.nch, ch = blockIdx.x % p.nch;
-    if (u >= p.ucount[bh]) return;
-    const int64_t j = p.ulist[bh * p.umax + u];
-    const uint32_t mask = p.umask[bh * p.umax + u];
-    const int64_t bend = (j == p.c) ? p.L : (j + 1) * p.bs;  // keys [j*bs, bend)
-    const int64_t k0 = j * p.bs + ch * p.chunk;
-    const int64_t k1 = (k0 + p.chunk < bend) ? k0 + p.chunk : bend;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g8 = lane >> 2, t4 = lane & 3;
     const int G = p.G;
-    // this warp's keys [kw0, kw1): a quarter of the chunk, in stages of 16
-    const int64_t wk = p.chunk / DEC_WARPS;
-    const int64_t kw0 = k0 + warp * wk;
-    const int64_t kw1 = (kw0 + wk < k1) ? kw0 + wk : (k1 > kw0 ? k1 : kw0);
-    const int nst = (int)((kw1 - kw0 + DEC_SKEYS - 1) / DEC_SKEYS);
-
-    // Q as A fragments, 8 steps of 16 features
+    dec_allow_dependents();
+    // Q as A fragments, 8 steps of 16 features (the caller's input: read before the wait)
     uint32_t qa[8][4];
     {
         const uint16_t* qb = p.q + ((int64_t)b * p.Hq + (int64_t)hk * G) * MOBA_D;
@@ -308,6 +308,19 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 2) moba_decode_attend_kernel(c
             qa[ks][3] = g8 + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (g8 + 8) * MOBA_D + f + 8) : 0u;
         }
     }
+    dec_wait_prior_grid();  // the union
+    if (u >= p.ucount[bh]) return;
+    const int64_t j = p.ulist[bh * p.umax + u];
+    const uint32_t mask = p.umask[bh * p.umax + u];
+    const int64_t bend = (j == p.c) ? p.L : (j + 1) * p.bs;  // keys [j*bs, bend)
+    const int64_t k0 = j * p.bs + ch * p.chunk;
+    const int64_t k1 = (k0 + p.chunk < bend) ? k0 + p.chunk : bend;
+    // this warp's keys [kw0, kw1): a quarter of the chunk, in stages of 16
+    const int64_t wk = p.chunk / DEC_WARPS;
+    const int64_t kw0 = k0 + warp * wk;
+    const int64_t kw1 = (kw0 + wk < k1) ? kw0 + wk : (k1 > kw0 ? k1 : kw0);
+    const int nst = (int)((kw1 - kw0 + DEC_SKEYS - 1) / DEC_SKEYS);
+
     uint8_t* ring = smem + warp * (DEC_STAGES * DEC_STAGE_BYTES);
     // stage s of this warp: 16 keys of K then of V in 16-byte chunks, rows past kw1 zero-filled;
     // one commit for every stage number (empty past the last) keeps the group count uniform
@@ -477,6 +490,7 @@ __global__ void __launch_bounds__(DEC_MERGE_THREADS) moba_decode_merge_kernel(co
     const int hq = blockIdx.x, b = blockIdx.y;
     const int hk = hq / p.G, g = hq % p.G;
     const int64_t bh = (int64_t)b * p.Hkv + hk;
+    dec_wait_prior_grid();  // the attend partials
     const int64_t total = (int64_t)p.ucount[bh] * p.nch;  // partial i: union entry i / nch, chunk i % nch
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const float* base = p.part + bh * p.umax * p.nch * (int64_t)p.G * DEC_PART + (int64_t)g * DEC_PART;

@@ -1022,6 +1022,24 @@ int make_decode_plan(int B, int Hq, int Hkv, int64_t L, int d, int bs, int topk,
 }
 
 
+// Launch of a decode kernel as a programmatic dependent of the kernel before it on the stream:
+// its CTAs may start while that kernel finishes, and wait for its results in griddepcontrol.wait.
+template <typename Kernel>
+cudaError_t launch_dependent(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             const DecodeParams& p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 }  // namespace
 
 extern "C" int moba_decode_workspace_size(int B, int Hq, int Hkv, int64_t L, int d, int block_size, int topk,
@@ -1138,7 +1156,11 @@ extern "C" int moba_decode(const void* q, const void* k, const void* v, const do
                 rc = cuda_fail(e);
                 break;
             }
-            moba_decode_union_kernel<<<dim3(Hkv, B), DEC_UNION_THREADS, smem_union, st>>>(p);
+            e = launch_dependent(moba_decode_union_kernel, dim3(Hkv, B), dim3(DEC_UNION_THREADS), smem_union, st, p);
+            if (e != cudaSuccess) {
+                rc = cuda_fail(e);
+                break;
+            }
             count_launch();
             if ((rc = launch_ok())) break;
         }
@@ -1150,11 +1172,21 @@ extern "C" int moba_decode(const void* q, const void* k, const void* v, const do
                 break;
             }
             dim3 grid((unsigned)(p.umax * p.nch), Hkv, B);
-            moba_decode_attend_kernel<<<grid, DEC_WARPS * 32, DEC_ATTEND_SMEM, st>>>(p);
+            e = launch_dependent(moba_decode_attend_kernel, grid, dim3(DEC_WARPS * 32), DEC_ATTEND_SMEM, st, p);
+            if (e != cudaSuccess) {
+                rc = cuda_fail(e);
+                break;
+            }
             count_launch();
             if ((rc = launch_ok())) break;
         }
-        moba_decode_merge_kernel<<<dim3(Hq, B), DEC_MERGE_THREADS, 0, st>>>(p);
+        {
+            const cudaError_t e = launch_dependent(moba_decode_merge_kernel, dim3(Hq, B), dim3(DEC_MERGE_THREADS), 0, st, p);
+            if (e != cudaSuccess) {
+                rc = cuda_fail(e);
+                break;
+            }
+        }
         count_launch();
         rc = launch_ok();
     } while (0);
